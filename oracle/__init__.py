@@ -1,0 +1,211 @@
+"""CPU oracle for fine-grained FP8 quantisation and the block-scaled FP8 GEMM.
+
+TEST INFRASTRUCTURE ONLY: only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline
+leg of ``bench.py`` may import this package.  It shares no code with the CUDA path
+(``fp8_fine_grained_fp8q_b200``) and neither imports the other.
+
+What it computes, from the pages on the DeepSeek-V3 Technical Report (arXiv 2412.19437):
+
+* E4M3 codes for every FP8 operand -- "DeepSeek-V3 Technical Report" summary page
+  (xyznot.com), Key ideas, FP8 mixed-precision bullet; Questions, the answer on training FP8
+  without divergence.
+* 1x128 tile-wise activation scales and 128x128 block-wise weight scales -- same passages.
+* 128x1 (token-direction) scales for the Wgrad operands: the groups run along the GEMM's inner
+  dimension -- DeepSeek-V3 report repost (why-be.co.kr), paragraph 4; Wgrad runs in FP8 --
+  paragraph 2 (Figure 6) and paragraph 3.
+* The GEMM D = sum_k A(m,k) B(k,n) of the dequantised operands, with the per-128-K scales
+  applied to each 128-wide partial sum at promotion -- repost paragraphs 1 and 4 (N_c = 128,
+  Figure 7(b)); summary page FP8 bullet.  Mathematically that equals the plain dot product of
+  the dequantised operands, which is what the oracle evaluates, exactly in binary64.
+  Fprop and Dgrad outputs are bf16, the Wgrad output FP32 (repost paragraph 3: gradients in
+  FP32).
+
+Readings the pages leave open (OCP E4M3FN, round-to-nearest-even with saturation at 448,
+max-abs scaling with an amax floor of 2^-100) are stated in ``fp8q_oracle.c``.
+
+The arithmetic lives in ``fp8q_oracle.c``; this module only marshals numpy arrays.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+FPROP, DGRAD, WGRAD = 0, 1, 2
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        I64 = ctypes.c_int64
+        lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+        lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        lib.oracle_e4m3_decode.restype = ctypes.c_double
+        lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_encode_array.argtypes = [P, I64, P]
+        lib.oracle_e4m3_decode_array.argtypes = [P, I64, P]
+        lib.oracle_quant_1x128.argtypes = [P, I64, I64, P, P]
+        lib.oracle_quant_128x1_t.argtypes = [P, I64, I64, P, P]
+        lib.oracle_quant_128x128.argtypes = [P, I64, I64, P, P, P]
+        lib.oracle_gemm.argtypes = [ctypes.c_int, P, P, P, P, I64, I64, I64, P, P, P, P]
+        lib.oracle_gemm_entries.argtypes = [ctypes.c_int, P, P, P, P, I64, I64, I64, P, P,
+                                            I64, P, P]
+        lib.oracle_grouped_entries.argtypes = [P, P, P, P, P, ctypes.c_int32, I64, I64, I64,
+                                               P, P, I64, P, P]
+        lib.oracle_num_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray) -> int:
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return a.ctypes.data
+
+
+def _bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Accept bf16 payloads as uint16 bit patterns (the seeded generators produce these)."""
+    x = np.ascontiguousarray(x)
+    if x.dtype != np.uint16:
+        raise TypeError("bf16 inputs are passed as uint16 bit patterns")
+    return x
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+# ----------------------------------------------------------------------------------------- #
+# E4M3 codec
+# ----------------------------------------------------------------------------------------- #
+
+def e4m3_encode(x) -> np.ndarray:
+    """E4M3FN codes of binary32 values: round to nearest even, saturate at +-448."""
+    x = np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+    out = np.empty(x.shape, dtype=np.uint8)
+    _load().oracle_e4m3_encode_array(_ptr(x), x.size, _ptr(out))
+    return out
+
+
+def e4m3_decode(c) -> np.ndarray:
+    """Exact binary64 values of E4M3FN codes (NaN for 0x7F / 0xFF)."""
+    c = np.ascontiguousarray(np.asarray(c, dtype=np.uint8))
+    out = np.empty(c.shape, dtype=np.float64)
+    _load().oracle_e4m3_decode_array(_ptr(c), c.size, _ptr(out))
+    return out
+
+
+# ----------------------------------------------------------------------------------------- #
+# Quantisers
+# ----------------------------------------------------------------------------------------- #
+
+def quant_1x128(x_bits: np.ndarray):
+    """x[M,K] bf16 bits -> (q[M,K] uint8, s[K/128, M] float32)."""
+    x = _bf16_bits(x_bits)
+    M, K = x.shape
+    q = np.empty((M, K), dtype=np.uint8)
+    s = np.empty((K // 128, M), dtype=np.float32)
+    _load().oracle_quant_1x128(_ptr(x), M, K, _ptr(q), _ptr(s))
+    return q, s
+
+
+def quant_128x1_t(x_bits: np.ndarray):
+    """x[T,C] bf16 bits -> (qt[C,T] uint8, s[T/128, C] float32)."""
+    x = _bf16_bits(x_bits)
+    T, C = x.shape
+    qt = np.empty((C, T), dtype=np.uint8)
+    s = np.empty((T // 128, C), dtype=np.float32)
+    _load().oracle_quant_128x1_t(_ptr(x), T, C, _ptr(qt), _ptr(s))
+    return qt, s
+
+
+def quant_128x128(w_bits: np.ndarray, want_transposed: bool = False):
+    """w[N,K] bf16 bits -> (q[N,K], s[N/128, K/128], qt[K,N] or None)."""
+    w = _bf16_bits(w_bits)
+    N, K = w.shape
+    q = np.empty((N, K), dtype=np.uint8)
+    s = np.empty((N // 128, K // 128), dtype=np.float32)
+    qt = np.empty((K, N), dtype=np.uint8) if want_transposed else None
+    _load().oracle_quant_128x128(_ptr(w), N, K, _ptr(q), _ptr(s),
+                                 _ptr(qt) if qt is not None else None)
+    return q, s, qt
+
+
+# ----------------------------------------------------------------------------------------- #
+# GEMM
+# ----------------------------------------------------------------------------------------- #
+
+def _gemm_dims(mode, A, B):
+    M, K = A.shape
+    if mode == DGRAD:
+        Kb, N = B.shape
+    else:
+        N, Kb = B.shape
+    assert Kb == K, "inner dimensions differ"
+    return M, N, K
+
+
+def gemm(mode: int, A, sA, B, sB):
+    """Exact binary64 D[M,N] and S[M,N] = sum_k |A(m,k) B(k,n)| of the dequantised operands.
+
+    A: [M,K] codes, sA: [K/128, M].  B and sB per mode:
+    FPROP  B = W[N,K],  sB = [N/128, K/128]
+    DGRAD  B = W[K,N] (the forward weight, used transposed), sB = [K/128, N/128]
+    WGRAD  B = X^T[N,K], sB = [K/128, N]
+    """
+    A = np.ascontiguousarray(A, dtype=np.uint8)
+    B = np.ascontiguousarray(B, dtype=np.uint8)
+    sA = np.ascontiguousarray(sA, dtype=np.float32)
+    sB = np.ascontiguousarray(sB, dtype=np.float32)
+    M, N, K = _gemm_dims(mode, A, B)
+    D = np.empty((M, N), dtype=np.float64)
+    S = np.empty((M, N), dtype=np.float64)
+    wa = np.empty((M, K), dtype=np.float64)
+    wb = np.empty((N, K), dtype=np.float64)
+    _load().oracle_gemm(mode, _ptr(A), _ptr(sA), _ptr(B), _ptr(sB), M, N, K,
+                        _ptr(D), _ptr(S), _ptr(wa), _ptr(wb))
+    return D, S
+
+
+def gemm_entries(mode: int, A, sA, B, sB, ms, ns):
+    """D[ms[i], ns[i]] and S[ms[i], ns[i]] only (for full-size problems)."""
+    A = np.ascontiguousarray(A, dtype=np.uint8)
+    B = np.ascontiguousarray(B, dtype=np.uint8)
+    sA = np.ascontiguousarray(sA, dtype=np.float32)
+    sB = np.ascontiguousarray(sB, dtype=np.float32)
+    M, N, K = _gemm_dims(mode, A, B)
+    ms = np.ascontiguousarray(ms, dtype=np.int64)
+    ns = np.ascontiguousarray(ns, dtype=np.int64)
+    assert ms.shape == ns.shape
+    out = np.empty(ms.shape, dtype=np.float64)
+    sabs = np.empty(ms.shape, dtype=np.float64)
+    _load().oracle_gemm_entries(mode, _ptr(A), _ptr(sA), _ptr(B), _ptr(sB), M, N, K,
+                                _ptr(ms), _ptr(ns), ms.size, _ptr(out), _ptr(sabs))
+    return out, sabs
+
+
+def grouped_entries(A, sA, B, sB, offsets, ms, ns):
+    """Grouped Fprop entries: A[Mtot,K], sA[K/128,Mtot], B[E,N,K], sB[E,N/128,K/128],
+    offsets[E+1] (rows of expert e are offsets[e]..offsets[e+1]-1)."""
+    A = np.ascontiguousarray(A, dtype=np.uint8)
+    B = np.ascontiguousarray(B, dtype=np.uint8)
+    sA = np.ascontiguousarray(sA, dtype=np.float32)
+    sB = np.ascontiguousarray(sB, dtype=np.float32)
+    off = np.ascontiguousarray(offsets, dtype=np.int32)
+    Mtot, K = A.shape
+    E, N, Kb = B.shape
+    assert Kb == K and off.size == E + 1
+    ms = np.ascontiguousarray(ms, dtype=np.int64)
+    ns = np.ascontiguousarray(ns, dtype=np.int64)
+    out = np.empty(ms.shape, dtype=np.float64)
+    sabs = np.empty(ms.shape, dtype=np.float64)
+    _load().oracle_grouped_entries(_ptr(A), _ptr(sA), _ptr(B), _ptr(sB), _ptr(off), E, Mtot,
+                                   N, K, _ptr(ms), _ptr(ns), ms.size, _ptr(out), _ptr(sabs))
+    return out, sabs
