@@ -1,0 +1,450 @@
+#!/usr/bin/env python
+"""Benchmark: one FP8 linear layer's training GEMMs on B200 through libfp8q.
+
+Workload (one "step"): the DeepSeek-V3 expert-FFN up-projection linear layer with 4096 tokens,
+C_in = 7168, C_out = 2048, bf16 operands resident in HBM:
+    act 1x128 (X)  -> weight 128x128 (W) -> Fprop  Y  = X W^T      (bf16 [4096, 2048])
+    act 1x128 (dY)                      -> Dgrad  dX = dY W        (bf16 [4096, 7168])
+    act 128x1^T (X), act 128x1^T (dY)   -> Wgrad  dW = dY^T X      (fp32 [2048, 7168])
+8 kernel launches.  value = GEMM FLOPs (3 x 2*4096*2048*7168) / device time of the step.
+L2 is flushed (256 MiB write) between steps, outside the timed step.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own replica of the step
+(weak scaling, no data-path collective); the step time is the max over ranks.
+--impl reference times the CPU oracle on a bounded slice of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+T_TOK, C_IN, C_OUT = 4096, 7168, 2048
+GEMM_FLOP = 2.0 * T_TOK * C_OUT * C_IN           # each of Fprop, Dgrad, Wgrad
+STEP_FLOP = 3.0 * GEMM_FLOP
+METRIC = ("block-scaled FP8 GEMM TFLOP/s (% dense FP8 peak); quantizer GB/s (% HBM)")
+WORKLOAD = ("FP8 linear layer training GEMMs (act 1x128 + weight 128x128 + Fprop, act 1x128 + "
+            "Dgrad, 2x act 128x1-transposed + Wgrad), tokens 4096, C_in 7168, C_out 2048")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP8_OVER_BF16 = 2.0                              # nominal dense ratio (4.5 / 2.25 PFLOP/s)
+
+# Algorithmic bytes per element: bf16 read (2) + code write (1) + one fp32 scale per group.
+QB_1x128 = 2 + 1 + 4 / 128
+QB_128x128 = 2 + 1 + 4 / (128 * 128)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "fp8_fine_grained_fp8q_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if taken on this source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if d.get("source_hash") != source_hash():
+        return None
+    return d
+
+
+# ------------------------------------------------------------------------------------------ #
+# Clock sampling (read-only NVML queries)
+# ------------------------------------------------------------------------------------------ #
+class ClockSampler:
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nvml = None
+
+    def _run(self):
+        nv = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit and bit != 0x1:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------------------------------ #
+# GPU arm
+# ------------------------------------------------------------------------------------------ #
+OPS = ["act_1x128_X", "weight_128x128_W", "gemm_fprop", "act_1x128_dY", "gemm_dgrad",
+       "act_128x1t_X", "act_128x1t_dY", "gemm_wgrad"]
+
+
+def make_buffers(torch, dev):
+    from fp8_fine_grained_fp8q_b200 import synth
+    d = synth.linear_layer(T_TOK, C_IN, C_OUT)
+    host = {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).pin_memory()
+            for k, v in d.items()}
+    t = {k: v.to(dev, non_blocking=False) for k, v in host.items()}
+    u8, f32, bf16 = torch.uint8, torch.float32, torch.bfloat16
+    e = lambda shape, dt: torch.empty(shape, dtype=dt, device=dev)  # noqa: E731
+    b = {
+        "Xq": e((T_TOK, C_IN), u8), "sX": e((C_IN // 128, T_TOK), f32),
+        "Wq": e((C_OUT, C_IN), u8), "sW": e((C_OUT // 128, C_IN // 128), f32),
+        "Y": e((T_TOK, C_OUT), bf16),
+        "dYq": e((T_TOK, C_OUT), u8), "sdY": e((C_OUT // 128, T_TOK), f32),
+        "dX": e((T_TOK, C_IN), bf16),
+        "Xtq": e((C_IN, T_TOK), u8), "sXt": e((T_TOK // 128, C_IN), f32),
+        "dYtq": e((C_OUT, T_TOK), u8), "sdYt": e((T_TOK // 128, C_OUT), f32),
+        "dW": e((C_OUT, C_IN), f32),
+    }
+    return host, t, b
+
+
+def step_ops(ops, t, b):
+    """The step as a list of zero-argument launches (all on torch's current stream)."""
+    return [
+        lambda: ops.act_1x128(t["X"], b["Xq"], b["sX"]),
+        lambda: ops.weight_128x128(t["W"], b["Wq"], b["sW"]),
+        lambda: ops.gemm_blockscaled(ops.FPROP, b["Xq"], b["sX"], b["Wq"], b["sW"], b["Y"]),
+        lambda: ops.act_1x128(t["dY"], b["dYq"], b["sdY"]),
+        lambda: ops.gemm_blockscaled(ops.DGRAD, b["dYq"], b["sdY"], b["Wq"], b["sW"], b["dX"]),
+        lambda: ops.act_128x1_transposed(t["X"], b["Xtq"], b["sXt"]),
+        lambda: ops.act_128x1_transposed(t["dY"], b["dYtq"], b["sdYt"]),
+        lambda: ops.gemm_blockscaled(ops.WGRAD, b["dYtq"], b["sdYt"], b["Xtq"], b["sXt"], b["dW"]),
+    ]
+
+
+def op_work():
+    """Algorithmic work per launch: ('flop', F) or ('bytes', B)."""
+    return {
+        "act_1x128_X": ("bytes", T_TOK * C_IN * QB_1x128),
+        "weight_128x128_W": ("bytes", C_OUT * C_IN * QB_128x128),
+        "gemm_fprop": ("flop", GEMM_FLOP),
+        "act_1x128_dY": ("bytes", T_TOK * C_OUT * QB_1x128),
+        "gemm_dgrad": ("flop", GEMM_FLOP),
+        "act_128x1t_X": ("bytes", T_TOK * C_IN * QB_1x128),
+        "act_128x1t_dY": ("bytes", T_TOK * C_OUT * QB_1x128),
+        "gemm_wgrad": ("flop", GEMM_FLOP),
+    }
+
+
+def run_ours(args, rank, world, dist):
+    import torch
+    from fp8_fine_grained_fp8q_b200 import ops
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ops.lib()                                      # fail loudly if the library is missing
+    host, t, b = make_buffers(torch, dev)
+    launches = step_ops(ops, t, b)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        for f in launches:
+            f()
+    torch.cuda.synchronize()
+    status = ops.device_status(dev)
+    if status != ops.DEV_OK:
+        raise RuntimeError(f"device status {status} after warm-up")
+
+    n_ev = len(launches) + 1
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        start.record()
+        for s in range(args.steps):
+            flush.zero_()
+            evs[s][0].record()
+            for i, f in enumerate(launches):
+                f()
+                evs[s][i + 1].record()
+        end.record()
+        torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    status = ops.device_status(dev)
+    if status != ops.DEV_OK:
+        raise RuntimeError(f"device status {status} in the timed region")
+
+    per_op = {name: [] for name in OPS}
+    step_ms = []
+    for s in range(args.steps):
+        step_ms.append(evs[s][0].elapsed_time(evs[s][-1]))
+        for i, name in enumerate(OPS):
+            per_op[name].append(evs[s][i].elapsed_time(evs[s][i + 1]))
+    sum_step_ms = float(sum(step_ms))
+    total_ms = start.elapsed_time(end)
+    if dist is not None:
+        tt = torch.tensor([sum_step_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        sum_step_ms = float(tt.item())
+    ms_per_step = sum_step_ms / args.steps
+    value = world * STEP_FLOP / (ms_per_step * 1e-3) / 1e12
+
+    # End to end through the same public calls, host buffers: H2D of this step's inputs from
+    # pinned memory, the step, D2H of its outputs, all in the timed region.
+    out_host = {k: torch.empty(b[k].shape, dtype=b[k].dtype, pin_memory=True)
+                for k in ("Y", "dX", "dW")}
+    e2e_steps = max(3, min(args.steps, 20))
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = sum(v.numel() * v.element_size() for v in out_host.values())
+    e2e_ms = []
+    for s in range(e2e_steps + 2):
+        flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for k in host:
+            t[k].copy_(host[k], non_blocking=True)
+        for f in launches:
+            f()
+        for k in out_host:
+            out_host[k].copy_(b[k], non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        if s >= 2:
+            e2e_ms.append(e0.elapsed_time(e1))
+    e2e_sum = float(sum(e2e_ms))
+    if dist is not None:
+        tt = torch.tensor([e2e_sum], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_sum = float(tt.item())
+    e2e_value = world * STEP_FLOP / (e2e_sum / len(e2e_ms) * 1e-3) / 1e12
+
+    peaks, peak_kind = load_peaks()
+    fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
+    hbm = peaks["hbm_gbs"]
+    work = op_work()
+    kernels = {}
+    for name in OPS:
+        ms = statistics.mean(per_op[name])
+        kind, amount = work[name]
+        if kind == "flop":
+            ach = amount / (ms * 1e-3) / 1e12
+            kernels[name] = {"ms": round(ms, 5), "TFLOP/s": round(ach, 1),
+                             "frac_fp8_peak": round(ach / fp8_peak, 4)}
+        else:
+            ach = amount / (ms * 1e-3) / 1e9
+            kernels[name] = {"ms": round(ms, 5), "GB/s": round(ach, 1),
+                             "frac_hbm": round(ach / hbm, 4)}
+    gemm_ms = statistics.mean([statistics.mean(per_op[n]) for n in ("gemm_fprop", "gemm_dgrad", "gemm_wgrad")])
+    gemm_ach = GEMM_FLOP / (gemm_ms * 1e-3) / 1e12
+    traffic = load_traffic()
+    roofline = {
+        "kernel": "gemm_blockscaled_kernel (fprop, dgrad, wgrad launches; 120.26 GFLOP each)",
+        "bound": "tensor", "achieved": round(gemm_ach, 1), "peak": round(fp8_peak, 1),
+        "unit": "TFLOP/s", "frac": round(gemm_ach / fp8_peak, 4),
+        "peak_source": f"{peak_kind} bf16 burst {peaks['bf16_tflops']} TFLOP/s x {FP8_OVER_BF16} "
+                       "(nominal dense FP8/BF16 ratio)",
+        "traffic": (traffic or {}).get("gemm_bytes_per_launch"),
+    }
+    q_ms = sum(statistics.mean(per_op[n]) for n in OPS if n.startswith(("act", "weight")))
+    q_bytes = sum(work[n][1] for n in OPS if n.startswith(("act", "weight")))
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8_e4m3 (fp32 accumulate)", "data": "synthetic (seeded)",
+        "config": {"workload": WORKLOAD, "tokens": T_TOK, "c_in": C_IN, "c_out": C_OUT,
+                   "l2": "flushed by a 256 MiB write before every step, outside the step",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "roofline": roofline,
+        "quantizers": {"GB/s": round(q_bytes / (q_ms * 1e-3) / 1e9, 1),
+                       "frac_hbm": round(q_bytes / (q_ms * 1e-3) / 1e9 / hbm, 4),
+                       "hbm_peak_gbs": hbm, "peak_source": peak_kind},
+        "kernels": kernels,
+        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h), "steps": len(e2e_ms)},
+        "gpu_launches": len(launches) * args.steps,
+        "clocks": clocks.summary(),
+        "wall_ms_timed_region": round(total_ms, 3),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_budget)
+    return line
+
+
+# ------------------------------------------------------------------------------------------ #
+# CPU oracle (baseline leg and --impl reference)
+# ------------------------------------------------------------------------------------------ #
+SLICE_T, SLICE_OUT = 128, 128
+
+
+def oracle_slice_inputs():
+    from fp8_fine_grained_fp8q_b200 import synth
+    d = synth.linear_layer(T_TOK, C_IN, C_OUT)
+    return {"X": np.ascontiguousarray(d["X"][:SLICE_T]),
+            "W": np.ascontiguousarray(d["W"][:SLICE_OUT]),
+            "dY": np.ascontiguousarray(d["dY"][:SLICE_T, :SLICE_OUT])}
+
+
+def oracle_step(oracle, d):
+    xq, xs = oracle.quant_1x128(d["X"])
+    wq, ws, _ = oracle.quant_128x128(d["W"])
+    oracle.gemm(oracle.FPROP, xq, xs, wq, ws)
+    gq, gs = oracle.quant_1x128(d["dY"])
+    oracle.gemm(oracle.DGRAD, gq, gs, wq, ws)
+    xtq, xts = oracle.quant_128x1_t(d["X"])
+    gtq, gts = oracle.quant_128x1_t(d["dY"])
+    oracle.gemm(oracle.WGRAD, gtq, gts, xtq, xts)
+
+
+SLICE_FLOP = 3 * 2.0 * SLICE_T * SLICE_OUT * C_IN
+SLICE_DESC = (f"the same step on a slice of the same layer: {SLICE_T} of 4096 tokens and "
+              f"{SLICE_OUT} of 2048 output channels, full C_in = 7168 (1/512 of the GEMM work); "
+              "value = GEMM FLOPs of the slice / oracle time")
+
+
+def cpu_baseline(budget_s: float = 15.0):
+    import oracle
+    d = oracle_slice_inputs()
+    oracle_step(oracle, d)                         # warm (and build) once
+    times = []
+    t_end = time.perf_counter() + budget_s
+    while time.perf_counter() < t_end or len(times) < 2:
+        t0 = time.perf_counter()
+        oracle_step(oracle, d)
+        times.append(time.perf_counter() - t0)
+    mean = statistics.mean(times)
+    return {"value": round(SLICE_FLOP / mean / 1e12, 6), "unit": "TFLOP/s",
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": SLICE_DESC + f"; {len(times)} repetitions, {sum(times):.1f} s"}
+
+
+def run_reference(args, rank, world):
+    import oracle
+    d = oracle_slice_inputs()
+    for _ in range(args.warmup):
+        oracle_step(oracle, d)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle_step(oracle, d)
+        times.append(time.perf_counter() - t0)
+    ms = statistics.mean(times) * 1e3
+    value = SLICE_FLOP / (ms * 1e-3) / 1e12
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)",
+        "config": {"workload": WORKLOAD, "tokens": T_TOK, "c_in": C_IN, "c_out": C_OUT,
+                   "sample": SLICE_DESC},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": SLICE_DESC},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle CPU work")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be at least 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        print(json.dumps(run_reference(args, rank, world)), flush=True)
+        return
+
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    try:
+        line = run_ours(args, rank, world, dist)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,321 @@
+// fp8q.cu -- the C ABI of libfp8q.so (declared in include/fp8q.h): argument checks, TMA
+// descriptor set-up and kernel launches.  Every call is asynchronous on the caller's stream
+// and allocates no device memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "fp8q.h"
+#include "gemm.cuh"
+#include "ptx.cuh"
+#include "quant.cuh"
+
+namespace {
+
+using namespace fp8q;
+
+constexpr int kMaxDevices = 64;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int sm_count()
+{
+    static int counts[kMaxDevices] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+    if (counts[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        counts[dev] = n;
+    }
+    return counts[dev];
+}
+
+int launch_status()
+{
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------------------------------
+// TMA descriptors (the driver entry point is fetched through the runtime, so the library has
+// no link-time dependency on libcuda).
+// ------------------------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// Row-major uint8 matrix [outer][inner] with 128-byte swizzled boxes of box_inner x box_outer.
+bool make_tmap_u8(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                  uint32_t box_outer)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {inner};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------------------------------
+// GEMM launch
+// ------------------------------------------------------------------------------------------
+template <int MODE, int BN, bool GROUPED>
+int prepare_kernel()
+{
+    using S = GemmShape<MODE, BN, GROUPED>;
+    static int ready[kMaxDevices] = {0};   // 1 ok, -1 unusable
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FP8Q_ERR_CUDA;
+    if (ready[dev] == 0) {
+        auto kern = gemm_blockscaled_kernel<MODE, BN, GROUPED>;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmemBytes) != cudaSuccess)
+            return FP8Q_ERR_CUDA;
+        cudaFuncAttributes attr;
+        if (cudaFuncGetAttributes(&attr, kern) != cudaSuccess) return FP8Q_ERR_CUDA;
+        // The register hand-over (setmaxnreg) needs the launch-time allocation it redistributes;
+        // never launch a build whose allocation is smaller.
+        ready[dev] = (attr.numRegs >= S::kRegsLaunch) ? 1 : -1;
+    }
+    return ready[dev] == 1 ? FP8Q_OK : FP8Q_ERR_UNSUPPORTED;
+}
+
+template <int MODE, int BN, bool GROUPED>
+int launch_gemm(const uint8_t* A, const float* sA, const uint8_t* B, const float* sB, void* D,
+                const int32_t* offsets, int E, int64_t M, int64_t N, int64_t K, cudaStream_t st)
+{
+    using S = GemmShape<MODE, BN, GROUPED>;
+    const int prep = prepare_kernel<MODE, BN, GROUPED>();
+    if (prep != FP8Q_OK) return prep;
+    CUtensorMap ta, tb;
+    if (!make_tmap_u8(&ta, A, (uint64_t)K, (uint64_t)M, 128, 128)) return FP8Q_ERR_CUDA;
+    if (MODE == kModeDgrad) {
+        if (!make_tmap_u8(&tb, B, (uint64_t)N, (uint64_t)K, 128, 128)) return FP8Q_ERR_CUDA;
+    } else {
+        const uint64_t rows = GROUPED ? (uint64_t)E * (uint64_t)N : (uint64_t)N;
+        if (!make_tmap_u8(&tb, B, (uint64_t)K, rows, 128, BN)) return FP8Q_ERR_CUDA;
+    }
+    GemmArgs a;
+    a.sA = sA;
+    a.sB = sB;
+    a.D = D;
+    a.offsets = offsets;
+    a.E = E;
+    a.M = (int32_t)M;
+    a.N = (int32_t)N;
+    a.KB = (int32_t)(K / 128);
+    const int sms = sm_count();
+    if (sms <= 0) return FP8Q_ERR_CUDA;
+    // Grouped: at most ceil(Mtot/128) + E row tiles (each group adds at most one partial tile).
+    const int64_t m_tiles = GROUPED ? (M + 127) / 128 + E : (M + 127) / 128;
+    const int64_t tiles = m_tiles * (N / BN);
+    const int grid = (int)(tiles < sms ? tiles : sms);
+    if (grid <= 0) return FP8Q_OK;
+    gemm_blockscaled_kernel<MODE, BN, GROUPED><<<grid, S::kThreads, S::kSmemBytes, st>>>(ta, tb, a);
+    return launch_status();
+}
+
+// Tile width: 256 unless 128-wide tiles finish in fewer waves of persistent CTAs.
+int choose_bn(int64_t M, int64_t N, int extra_m_tiles)
+{
+    const char* env = getenv("FP8Q_GEMM_BN");
+    if (env && (N % 256 == 0) && atoi(env) == 256) return 256;
+    if (env && atoi(env) == 128) return 128;
+    if (N % 256 != 0) return 128;
+    const int sms = sm_count() > 0 ? sm_count() : 148;
+    const int64_t mt = (M + 127) / 128 + extra_m_tiles;
+    const int64_t w256 = (mt * (N / 256) + sms - 1) / sms;   // waves of 256-wide tiles (cost 2 each)
+    const int64_t w128 = (mt * (N / 128) + sms - 1) / sms;   // waves of 128-wide tiles (cost 1 each)
+    return (2 * w256 <= w128) ? 256 : 128;
+}
+
+template <int MODE>
+int gemm_mode(const uint8_t* A, const float* sA, const uint8_t* B, const float* sB, void* D, int64_t M,
+              int64_t N, int64_t K, cudaStream_t st)
+{
+    if (choose_bn(M, N, 0) == 256)
+        return launch_gemm<MODE, 256, false>(A, sA, B, sB, D, nullptr, 1, M, N, K, st);
+    return launch_gemm<MODE, 128, false>(A, sA, B, sB, D, nullptr, 1, M, N, K, st);
+}
+
+// Waits on an mbarrier that nothing ever arrives on, so the bounded wait must expire, latch
+// FP8Q_DEV_TIMEOUT and return.  Exercises the kernels' timeout path without a hang or a fault.
+__global__ void selftest_wait_kernel(uint64_t limit_ns)
+{
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait_slow(smem_u32(&bar), 0, &abort_flag, limit_ns);
+}
+
+}  // namespace
+
+// ==========================================================================================
+// C ABI
+// ==========================================================================================
+extern "C" {
+
+const char* fp8q_status_string(int status)
+{
+    switch (status) {
+    case FP8Q_OK: return "ok";
+    case FP8Q_ERR_ARG: return "invalid argument";
+    case FP8Q_ERR_SHAPE: return "shape: a 128-group dimension is not a multiple of 128";
+    case FP8Q_ERR_ALIGN: return "a data pointer is not 16-byte aligned";
+    case FP8Q_ERR_CUDA: return "CUDA error";
+    case FP8Q_ERR_UNSUPPORTED: return "size or configuration not supported by this build";
+    case FP8Q_ERR_DEVICE: return "error reported by the device";
+    default: return "unknown status";
+    }
+}
+
+int fp8q_abi_version(void) { return 1; }
+
+int fp8q_act_1x128(const uint16_t* x, int64_t M, int64_t K, uint8_t* q, float* s, fp8q_stream_t stream)
+{
+    if (M < 0 || K < 0) return FP8Q_ERR_ARG;
+    if (K % 128 != 0) return FP8Q_ERR_SHAPE;
+    if (M == 0 || K == 0) return FP8Q_OK;
+    if (!x || !q || !s) return FP8Q_ERR_ARG;
+    if (!aligned16(x) || !aligned16(q) || !aligned16(s)) return FP8Q_ERR_ALIGN;
+    const int sms = sm_count();
+    if (sms <= 0) return FP8Q_ERR_CUDA;
+    constexpr int kUnr = 4;
+    const int64_t ntiles = M * (K / 128);
+    const int64_t want = (ntiles + 16 * kUnr - 1) / (16 * kUnr);   // blocks of 16 half-warps
+    const int64_t cap = (int64_t)sms * 8;
+    const int grid = (int)(want < cap ? want : cap);
+    act_1x128_kernel<kUnr><<<grid, 256, 0, (cudaStream_t)stream>>>(x, q, s, M, K);
+    return launch_status();
+}
+
+int fp8q_act_128x1_transposed(const uint16_t* x, int64_t T, int64_t C, uint8_t* qt, float* s,
+                              fp8q_stream_t stream)
+{
+    if (T < 0 || C < 0) return FP8Q_ERR_ARG;
+    if (T % 128 != 0 || C % 64 != 0) return FP8Q_ERR_SHAPE;
+    if (T == 0 || C == 0) return FP8Q_OK;
+    if (!x || !qt || !s) return FP8Q_ERR_ARG;
+    if (!aligned16(x) || !aligned16(qt) || !aligned16(s)) return FP8Q_ERR_ALIGN;
+    if (T / 128 > 65535 || C / 64 > 0x7FFFFFFF) return FP8Q_ERR_UNSUPPORTED;
+    const dim3 grid((unsigned)(C / 64), (unsigned)(T / 128));
+    act_128x1_t_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(x, qt, s, T, C);
+    return launch_status();
+}
+
+int fp8q_weight_128x128(const uint16_t* w, int64_t N, int64_t K, uint8_t* q, float* s, uint8_t* qt_or_null,
+                        fp8q_stream_t stream)
+{
+    if (N < 0 || K < 0) return FP8Q_ERR_ARG;
+    if (N % 128 != 0 || K % 128 != 0) return FP8Q_ERR_SHAPE;
+    if (N == 0 || K == 0) return FP8Q_OK;
+    if (!w || !q || !s) return FP8Q_ERR_ARG;
+    if (!aligned16(w) || !aligned16(q) || !aligned16(s) || !aligned16(qt_or_null)) return FP8Q_ERR_ALIGN;
+    if (N / 128 > 65535 || K / 128 > 0x7FFFFFFF) return FP8Q_ERR_UNSUPPORTED;
+    const dim3 grid((unsigned)(K / 128), (unsigned)(N / 128));
+    weight_128x128_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(w, q, s, qt_or_null, N, K);
+    return launch_status();
+}
+
+size_t fp8q_gemm_workspace_size(int mode, int64_t M, int64_t N, int64_t K)
+{
+    (void)mode;
+    (void)M;
+    (void)N;
+    (void)K;
+    return 0;
+}
+
+int fp8_gemm_blockscaled(int mode, const uint8_t* A, const float* sA, const uint8_t* B, const float* sB, void* D,
+                         int64_t M, int64_t N, int64_t K, void* workspace, size_t ws_bytes, fp8q_stream_t stream)
+{
+    (void)workspace;
+    (void)ws_bytes;
+    if (mode != FP8Q_FPROP && mode != FP8Q_DGRAD && mode != FP8Q_WGRAD) return FP8Q_ERR_ARG;
+    if (M < 0 || N < 0 || K < 0) return FP8Q_ERR_ARG;
+    if (N % 128 != 0 || K % 128 != 0) return FP8Q_ERR_SHAPE;
+    if (M == 0 || N == 0) return FP8Q_OK;
+    if (M >= (1ll << 31) || N >= (1ll << 31) || K >= (1ll << 31)) return FP8Q_ERR_UNSUPPORTED;
+    if (!A || !sA || !B || !sB || !D) return FP8Q_ERR_ARG;
+    if (!aligned16(A) || !aligned16(sA) || !aligned16(B) || !aligned16(sB) || !aligned16(D)) return FP8Q_ERR_ALIGN;
+    if (K == 0) {
+        // An empty contraction: D = 0.
+        const size_t bytes = (size_t)M * (size_t)N * (mode == FP8Q_WGRAD ? 4u : 2u);
+        return cudaMemsetAsync(D, 0, bytes, (cudaStream_t)stream) == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+    }
+    const cudaStream_t st = (cudaStream_t)stream;
+    switch (mode) {
+    case FP8Q_FPROP: return gemm_mode<kModeFprop>(A, sA, B, sB, D, M, N, K, st);
+    case FP8Q_DGRAD: return gemm_mode<kModeDgrad>(A, sA, B, sB, D, M, N, K, st);
+    default: return gemm_mode<kModeWgrad>(A, sA, B, sB, D, M, N, K, st);
+    }
+}
+
+int fp8_grouped_gemm_blockscaled(const uint8_t* A, const float* sA, const uint8_t* B, const float* sB,
+                                 const int32_t* offsets, int32_t E, int64_t Mtot, int64_t N, int64_t K, uint16_t* D,
+                                 fp8q_stream_t stream)
+{
+    if (E < 1 || Mtot < 0 || N < 0 || K < 0) return FP8Q_ERR_ARG;
+    if (E > 1024) return FP8Q_ERR_UNSUPPORTED;
+    if (N % 128 != 0 || K % 128 != 0) return FP8Q_ERR_SHAPE;
+    if (Mtot == 0 || N == 0) return FP8Q_OK;
+    if (Mtot >= (1ll << 31) || (int64_t)E * N >= (1ll << 31) || K >= (1ll << 31)) return FP8Q_ERR_UNSUPPORTED;
+    if (!A || !sA || !B || !sB || !D || !offsets) return FP8Q_ERR_ARG;
+    if (!aligned16(A) || !aligned16(sA) || !aligned16(B) || !aligned16(sB) || !aligned16(D)) return FP8Q_ERR_ALIGN;
+    if ((reinterpret_cast<uintptr_t>(offsets) & 3u) != 0) return FP8Q_ERR_ALIGN;
+    const cudaStream_t st = (cudaStream_t)stream;
+    if (K == 0) {
+        return cudaMemsetAsync(D, 0, (size_t)Mtot * (size_t)N * 2u, st) == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+    }
+    if (choose_bn(Mtot, N, E) == 256)
+        return launch_gemm<kModeFprop, 256, true>(A, sA, B, sB, D, offsets, E, Mtot, N, K, st);
+    return launch_gemm<kModeFprop, 128, true>(A, sA, B, sB, D, offsets, E, Mtot, N, K, st);
+}
+
+int fp8q_selftest_wait_timeout(uint64_t limit_ns, fp8q_stream_t stream)
+{
+    if (limit_ns == 0 || limit_ns > 2000000000ull) return FP8Q_ERR_ARG;
+    selftest_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(limit_ns);
+    return launch_status();
+}
+
+int fp8q_device_status(fp8q_stream_t stream, int* out)
+{
+    if (!out) return FP8Q_ERR_ARG;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return FP8Q_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, fp8q::g_status, sizeof(int)) != cudaSuccess) return FP8Q_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(fp8q::g_status, &zero, sizeof(int)) != cudaSuccess) return FP8Q_ERR_CUDA;
+    *out = v;
+    return FP8Q_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,391 @@
+// gemm.cuh -- block-scaled FP8 GEMM on the 5th-generation tensor cores (tcgen05), with the
+// per-128-K scales applied when each K group's partial sum is promoted into FP32.
+//
+// What it computes (DeepSeek-V3 report repost, paragraphs 1 and 4, Figure 7(b);
+// "DeepSeek-V3 Technical Report" summary page, Key ideas, FP8 bullet):
+//   for each 128-wide K group kb:  P = sum_{k in kb} qA[m,k] qB(k,n)        (tensor cores, FP32)
+//                                  acc[m,n] += P * sA[kb][m] * sB(kb, n)    (CUDA cores, FP32)
+//   D = acc  (bf16 for Fprop / Dgrad, FP32 for Wgrad).
+// The pages' H800 design runs two WGMMA warpgroups so one promotes while the other multiplies.
+// Here the overlap comes from the asynchronous tcgen05 pipeline instead:
+//   warp 0      TMA producer: A and B tiles (128-byte swizzled) into a STAGES-deep ring;
+//               for Wgrad also the per-column scales of each K group (bulk copy).
+//   warp 1      MMA issuer: 4 x tcgen05.mma (K = 32 each) per K group into one of two TMEM
+//               partial buffers (a fresh accumulation per group), then tcgen05.commit.
+//   warps 4-11  promotion: tcgen05.ld the partial of group kb while the tensor cores fill the
+//               other buffer, fold in the scales and accumulate in registers (each warp owns 32
+//               rows x BN/2 columns); after the last group, convert and store the tile.
+// The CTA is persistent (one per SM) and walks a static tile list, so the epilogue of one
+// tile overlaps the first MMAs of the next.  setmaxnreg moves registers from the producer /
+// MMA warpgroup (40 each) to the two promotion warpgroups (232 each).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "ptx.cuh"
+
+namespace fp8q {
+
+enum { kModeFprop = 0, kModeDgrad = 1, kModeWgrad = 2 };
+
+struct GemmArgs {
+    const float* sA;          // [KB][M]
+    const float* sB;          // Fprop [N/128][KB] (x E if grouped); Dgrad [KB][N/128]; Wgrad [KB][N]
+    void* D;                  // [M][N], bf16 (Fprop / Dgrad) or fp32 (Wgrad)
+    const int32_t* offsets;   // grouped only: device [E+1]
+    int32_t E;                // number of groups (1 unless grouped)
+    int32_t M;                // rows of A and D
+    int32_t N;
+    int32_t KB;               // K / 128
+};
+
+template <int MODE, int BN, bool GROUPED>
+struct GemmShape {
+    static constexpr int kBM = 128;
+    static constexpr int kBK = 128;
+    static constexpr int kABytes = kBM * kBK;
+    static constexpr int kBBytes = BN * kBK;
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kStages = (BN == 256) ? 4 : 6;
+    static constexpr int kScaleStages = (MODE == kModeWgrad) ? 4 : 0;
+    static constexpr int kHalf = BN / 2;           // columns per promotion warp
+    static constexpr int kTmemCols = 2 * BN;       // two partial buffers
+    static constexpr int kThreads = 384;
+    static constexpr int kMaxGroups = 1024;
+    static constexpr int kOffScales = kStages * kStageBytes;
+    static constexpr int kOffBars = kOffScales + kScaleStages * BN * 4;
+    static constexpr int kNumBars = 2 * kStages + 4 + 2 * kScaleStages + 1;
+    static constexpr int kOffMisc = kOffBars + kNumBars * 8;
+    static constexpr int kOffGroups = kOffMisc + 16;
+    static constexpr int kSmemBytes = kOffGroups + (GROUPED ? 2 * (kMaxGroups + 1) * 4 : 0) + 1024;
+    // Registers: launched at 168 per thread (384 x 168 = 64512); 128 x 40 + 256 x 232 = 64512.
+    static constexpr int kRegsLow = 40;
+    static constexpr int kRegsHigh = 232;
+    static constexpr int kRegsLaunch = 168;
+    static_assert(kThreads * kRegsLaunch >= 128 * kRegsLow + 256 * kRegsHigh, "register split");
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+};
+
+struct TileInfo {
+    int32_t row0;      // first row of the 128-row tile
+    int32_t row_end;   // rows >= row_end are not part of this tile's group (masked)
+    int32_t n0;        // first column
+    int32_t e;         // group
+};
+
+template <bool GROUPED>
+__device__ __forceinline__ TileInfo decode_tile(int t, int nb_tiles, int bn, const GemmArgs& a,
+                                                const int32_t* g_off, const int32_t* g_pre)
+{
+    const int mt = t / nb_tiles;
+    const int nt = t - mt * nb_tiles;
+    TileInfo ti;
+    ti.n0 = nt * bn;
+    if (GROUPED) {
+        int lo = 0, hi = a.E;   // g_pre[lo] <= mt < g_pre[hi]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (g_pre[mid] <= mt) lo = mid; else hi = mid;
+        }
+        ti.e = lo;
+        ti.row0 = g_off[lo] + (mt - g_pre[lo]) * 128;
+        ti.row_end = g_off[lo + 1];
+    } else {
+        ti.e = 0;
+        ti.row0 = mt * 128;
+        ti.row_end = a.M;
+    }
+    return ti;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+template <int MODE, int BN, bool GROUPED>
+__global__ void __launch_bounds__(384, 1)
+gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const GemmArgs args)
+{
+    using S = GemmShape<MODE, BN, GROUPED>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float* col_scales = reinterpret_cast<float*>(smem + S::kOffScales);
+    uint32_t* misc = reinterpret_cast<uint32_t*>(smem + S::kOffMisc);   // [0] TMEM base, [1] abort, [2] bad groups
+    int32_t* g_off = reinterpret_cast<int32_t*>(smem + S::kOffGroups);
+    int32_t* g_pre = g_off + (S::kMaxGroups + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+
+    const uint32_t bar0 = smem_u32(smem + S::kOffBars);
+    const auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    const auto empty_bar = [&](int s) { return bar0 + 8u * (S::kStages + s); };
+    const auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * S::kStages + b); };
+    const auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * S::kStages + 2 + b); };
+    const auto sfull_bar = [&](int s) { return bar0 + 8u * (2 * S::kStages + 4 + s); };
+    const auto sempty_bar = [&](int s) { return bar0 + 8u * (2 * S::kStages + 4 + S::kScaleStages + s); };
+    const uint32_t drain_bar = bar0 + 8u * (2 * S::kStages + 4 + 2 * S::kScaleStages);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // ---------------------------------------------------------------- set-up
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S::kStages; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(tfull_bar(b), 1);
+            mbar_init(tempty_bar(b), 8);
+        }
+        for (int s = 0; s < S::kScaleStages; ++s) {
+            mbar_init(sfull_bar(s), 1);
+            mbar_init(sempty_bar(s), 8);
+        }
+        mbar_init(drain_bar, 1);
+        misc[1] = 0;
+        misc[2] = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tmA);
+        prefetch_tensormap(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(misc), S::kTmemCols);
+        tmem_relinquish();
+    }
+    if (GROUPED && warp == 2) {
+        // Copy the offsets, validate them and build the prefix of 128-row tiles per group with a
+        // warp scan (each lane owns a contiguous run of groups).
+        const int E = args.E;
+        for (int i = lane; i <= E; i += 32) g_off[i] = __ldg(args.offsets + i);
+        __syncwarp();
+        const int per = (E + 31) >> 5;
+        const int lo = min(E, lane * per), hi = min(E, lo + per);
+        int local = 0;
+        bool bad = false;
+        for (int e = lo; e < hi; ++e) {
+            const int cnt = g_off[e + 1] - g_off[e];
+            bad |= cnt < 0;
+            local += cnt > 0 ? (cnt + 127) >> 7 : 0;
+        }
+        int incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        int run = incl - local;
+        for (int e = lo; e < hi; ++e) {
+            g_pre[e] = run;
+            const int cnt = g_off[e + 1] - g_off[e];
+            run += cnt > 0 ? (cnt + 127) >> 7 : 0;
+        }
+        if (lane == 31) g_pre[E] = incl;
+        if (lane == 0) bad |= (g_off[0] != 0) || (g_off[E] != args.M);
+        bad = __any_sync(0xFFFFFFFFu, bad);
+        if (bad && lane == 0) {
+            misc[2] = 1;
+            latch_status(2 /* FP8Q_DEV_BAD_OFFSETS */);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    const uint32_t tmem_base = misc[0];
+    const int nb_tiles = args.N / BN;
+    const int num_m_tiles = GROUPED ? (misc[2] ? 0 : g_pre[args.E]) : (args.M + 127) / 128;
+    const int num_tiles = num_m_tiles * nb_tiles;
+    const int KB = args.KB;
+
+    if (warp < 4) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(S::kRegsLow));
+        if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0, ss = 0;
+            uint32_t phase = 0, sph = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
+                const TileInfo ti = decode_tile<GROUPED>(t, nb_tiles, BN, args, g_off, g_pre);
+                const int brow = GROUPED ? ti.e * args.N + ti.n0 : ti.n0;
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) { ok = false; break; }
+                    const uint32_t sa = smem_u32(smem + stage * S::kStageBytes);
+                    const uint32_t sb = sa + S::kABytes;
+                    mbar_arrive_expect_tx(full_bar(stage), S::kStageBytes);
+                    tma_load_2d(sa, &tmA, kb * 128, ti.row0, full_bar(stage));
+                    if (MODE == kModeDgrad) {
+#pragma unroll
+                        for (int h = 0; h < BN / 128; ++h)
+                            tma_load_2d(sb + h * 16384, &tmB, ti.n0 + h * 128, kb * 128, full_bar(stage));
+                    } else {
+                        tma_load_2d(sb, &tmB, kb * 128, brow, full_bar(stage));
+                    }
+                    if (MODE == kModeWgrad) {
+                        if (!mbar_wait(sempty_bar(ss), sph ^ 1u, abort_flag)) { ok = false; break; }
+                        mbar_arrive_expect_tx(sfull_bar(ss), BN * 4);
+                        bulk_load(smem_u32(col_scales + ss * BN), args.sB + (size_t)kb * args.N + ti.n0, BN * 4,
+                                  sfull_bar(ss));
+                        if (++ss == S::kScaleStages) { ss = 0; sph ^= 1u; }
+                    }
+                    if (++stage == S::kStages) { stage = 0; phase ^= 1u; }
+                }
+            }
+            if (!ok) {
+                // Aborting: give copies already in flight time to land before the CTA exits.
+                const uint64_t t0 = globaltimer_ns();
+                while (globaltimer_ns() - t0 < 50000ull) __nanosleep(1000);
+            }
+        }
+        } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_e4m3_f32(BN, MODE == kModeDgrad);
+            int stage = 0, tb = 0;
+            uint32_t phase = 0, tph = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(tempty_bar(tb), tph ^ 1u, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait(full_bar(stage), phase, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(smem + stage * S::kStageBytes);
+                    const uint32_t sb = sa + S::kABytes;
+                    const uint32_t d = tmem_base + (uint32_t)(tb * BN);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint64_t ad = sdesc_sw128(sa + k * 32, 16, 1024);
+                        const uint64_t bd = (MODE == kModeDgrad) ? sdesc_sw128(sb + k * 4096, 16384, 1024)
+                                                                 : sdesc_sw128(sb + k * 32, 16, 1024);
+                        mma_f8f6f4(d, ad, bd, idesc, k > 0 ? 1u : 0u);
+                    }
+                    tc_commit(empty_bar(stage));
+                    tc_commit(tfull_bar(tb));
+                    if (++stage == S::kStages) { stage = 0; phase ^= 1u; }
+                    if (++tb == 2) { tb = 0; tph ^= 1u; }
+                }
+            }
+            // Drain: every MMA this thread issued has completed before TMEM is released.
+            tc_commit(drain_bar);
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(drain_bar, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+            }
+        }
+        __syncwarp();
+        // Release TMEM once the promotion warps have read their last partial.
+        named_bar_sync(1, 32 + 256);
+        tc_fence_after();
+        tmem_dealloc(tmem_base, S::kTmemCols);
+        }
+    } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(S::kRegsHigh));
+        // ------------------------------------------------------------ promotion + epilogue
+        const int pw = warp - 4;
+        const int quad = warp & 3;            // TMEM lanes 32*quad .. 32*quad+31
+        const int half = pw >> 2;             // columns [half*BN/2, (half+1)*BN/2)
+        const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+        const int rit = quad * 32 + lane;     // row within the tile
+        int tb = 0, ss = 0;
+        uint32_t tph = 0, sph = 0;
+        float acc[S::kHalf];
+        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+            const TileInfo ti = decode_tile<GROUPED>(t, nb_tiles, BN, args, g_off, g_pre);
+            const int row = ti.row0 + rit;
+            const bool in_a = row < args.M;
+            const int ncol0 = ti.n0 + half * S::kHalf;
+            const float* sa_ptr = args.sA + (in_a ? row : 0);
+            const float* sb_ptr = args.sB;
+            size_t sb_step = 0;
+            if (MODE == kModeFprop) {
+                sb_ptr = args.sB + (size_t)ti.e * (size_t)(args.N >> 7) * KB + (size_t)(ncol0 >> 7) * KB;
+                sb_step = 1;
+            } else if (MODE == kModeDgrad) {
+                sb_ptr = args.sB + (ncol0 >> 7);
+                sb_step = (size_t)(args.N >> 7);
+            }
+#pragma unroll
+            for (int i = 0; i < S::kHalf; ++i) acc[i] = 0.0f;
+            float sa_next = in_a ? __ldg(sa_ptr) : 0.0f;
+            float sb_next = (MODE != kModeWgrad) ? __ldg(sb_ptr) : 1.0f;
+            bool ok = true;
+            for (int kb = 0; kb < KB; ++kb) {
+                const float sa = sa_next, sbv = sb_next;
+                if (kb + 1 < KB) {
+                    sa_next = in_a ? __ldg(sa_ptr + (size_t)(kb + 1) * args.M) : 0.0f;
+                    if (MODE != kModeWgrad) sb_next = __ldg(sb_ptr + (size_t)(kb + 1) * sb_step);
+                }
+                if (!warp_wait(tfull_bar(tb), tph, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t taddr = tmem_base + lane_base + (uint32_t)(tb * BN + half * S::kHalf);
+                if (MODE != kModeWgrad) {
+                    const float c = sa * sbv;
+#pragma unroll
+                    for (int ch = 0; ch < S::kHalf / 32; ++ch) {
+                        float v[32];
+                        tmem_ld32(taddr + ch * 32, v);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) acc[ch * 32 + j] = fmaf(v[j], c, acc[ch * 32 + j]);
+                    }
+                } else {
+                    if (!warp_wait(sfull_bar(ss), sph, abort_flag)) { ok = false; break; }
+                    const float* cs = col_scales + ss * BN + half * S::kHalf;
+#pragma unroll
+                    for (int ch = 0; ch < S::kHalf / 32; ++ch) {
+                        float v[32];
+                        tmem_ld32(taddr + ch * 32, v);
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4) {
+                            const float4 c4 = *reinterpret_cast<const float4*>(cs + ch * 32 + j);
+                            acc[ch * 32 + j + 0] = fmaf(v[j + 0], sa * c4.x, acc[ch * 32 + j + 0]);
+                            acc[ch * 32 + j + 1] = fmaf(v[j + 1], sa * c4.y, acc[ch * 32 + j + 1]);
+                            acc[ch * 32 + j + 2] = fmaf(v[j + 2], sa * c4.z, acc[ch * 32 + j + 2]);
+                            acc[ch * 32 + j + 3] = fmaf(v[j + 3], sa * c4.w, acc[ch * 32 + j + 3]);
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(tempty_bar(tb));
+                    if (MODE == kModeWgrad) mbar_arrive(sempty_bar(ss));
+                }
+                if (MODE == kModeWgrad) {
+                    if (++ss == S::kScaleStages) { ss = 0; sph ^= 1u; }
+                }
+                if (++tb == 2) { tb = 0; tph ^= 1u; }
+            }
+            if (!ok) break;
+            // Epilogue: rows of this tile's group only.
+            if (row < ti.row_end) {
+                if (MODE == kModeWgrad) {
+                    float* drow = reinterpret_cast<float*>(args.D) + (size_t)row * args.N + ncol0;
+#pragma unroll
+                    for (int j = 0; j < S::kHalf; j += 4)
+                        *reinterpret_cast<float4*>(drow + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+                } else {
+                    uint16_t* drow = reinterpret_cast<uint16_t*>(args.D) + (size_t)row * args.N + ncol0;
+#pragma unroll
+                    for (int j = 0; j < S::kHalf; j += 8) {
+                        uint4 o;
+                        o.x = pack_bf16x2(acc[j + 0], acc[j + 1]);
+                        o.y = pack_bf16x2(acc[j + 2], acc[j + 3]);
+                        o.z = pack_bf16x2(acc[j + 4], acc[j + 5]);
+                        o.w = pack_bf16x2(acc[j + 6], acc[j + 7]);
+                        *reinterpret_cast<uint4*>(drow + j) = o;
+                    }
+                }
+            }
+        }
+        tc_fence_before();
+        named_bar_arrive(1, 32 + 256);
+    }
+
+}
+
+}  // namespace fp8q

@@ -1,0 +1,204 @@
+"""ctypes binding of libfp8q.so (C ABI in include/fp8q.h).
+
+Argument marshalling only: every step of the computation runs in the library's CUDA kernels.
+PyTorch provides device memory and the current stream.  There is no fallback path: if the
+library is missing or a call fails, an exception is raised.
+
+Tensor conventions (all CUDA, contiguous):
+  bf16 inputs are torch.bfloat16; E4M3 codes are torch.uint8 (view as torch.float8_e4m3fn if
+  wanted); scales are torch.float32 with the group-major layouts the header documents.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfp8q.so")
+
+FPROP, DGRAD, WGRAD = 0, 1, 2
+DEV_OK, DEV_TIMEOUT, DEV_BAD_OFFSETS = 0, 1, 2
+
+_lib = None
+
+
+class Fp8qError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {status_string(status)} (status {status})")
+
+
+def lib() -> ctypes.CDLL:
+    """Load libfp8q.so (built in-tree by fp8_fine_grained_fp8q_b200.build)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m fp8_fine_grained_fp8q_b200.build` (needs nvcc)")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I64, I32, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int
+    L.fp8q_status_string.restype = ctypes.c_char_p
+    L.fp8q_status_string.argtypes = [I]
+    L.fp8q_abi_version.restype = I
+    L.fp8q_abi_version.argtypes = []
+    for name, args in {
+        "fp8q_act_1x128": [P, I64, I64, P, P, P],
+        "fp8q_act_128x1_transposed": [P, I64, I64, P, P, P],
+        "fp8q_weight_128x128": [P, I64, I64, P, P, P, P],
+        "fp8_gemm_blockscaled": [I, P, P, P, P, P, I64, I64, I64, P, ctypes.c_size_t, P],
+        "fp8_grouped_gemm_blockscaled": [P, P, P, P, P, I32, I64, I64, I64, P, P],
+        "fp8q_device_status": [P, ctypes.POINTER(I)],
+    }.items():
+        fn = getattr(L, name)
+        fn.restype = I
+        fn.argtypes = args
+    L.fp8q_selftest_wait_timeout.restype = I
+    L.fp8q_selftest_wait_timeout.argtypes = [ctypes.c_uint64, P]
+    L.fp8q_gemm_workspace_size.restype = ctypes.c_size_t
+    L.fp8q_gemm_workspace_size.argtypes = [I, I64, I64, I64]
+    _lib = L
+    return L
+
+
+def status_string(status: int) -> str:
+    return lib().fp8q_status_string(int(status)).decode()
+
+
+def _stream(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise Fp8qError(fn, status)
+
+
+def _require(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions, got {t.dim()}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _out(t, shape, dtype, device, name):
+    if t is None:
+        return torch.empty(shape, dtype=dtype, device=device)
+    _require(t, name, dtype, len(shape))
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+def _p(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+# ------------------------------------------------------------------------------------------ #
+# Quantisers
+# ------------------------------------------------------------------------------------------ #
+
+def act_1x128(x: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tensor | None = None):
+    """x[M,K] bf16 -> (q[M,K] uint8 E4M3 codes, s[K/128, M] fp32)."""
+    _require(x, "x", torch.bfloat16, 2)
+    M, K = x.shape
+    q = _out(q, (M, K), torch.uint8, x.device, "q")
+    s = _out(s, (K // 128, M), torch.float32, x.device, "s")
+    _check("fp8q_act_1x128", lib().fp8q_act_1x128(_p(x), M, K, _p(q), _p(s), _stream(x.device)))
+    return q, s
+
+
+def act_128x1_transposed(x: torch.Tensor, qt: torch.Tensor | None = None,
+                         s: torch.Tensor | None = None):
+    """x[T,C] bf16 -> (qt[C,T] uint8, s[T/128, C] fp32)."""
+    _require(x, "x", torch.bfloat16, 2)
+    T, C = x.shape
+    qt = _out(qt, (C, T), torch.uint8, x.device, "qt")
+    s = _out(s, (T // 128, C), torch.float32, x.device, "s")
+    _check("fp8q_act_128x1_transposed",
+           lib().fp8q_act_128x1_transposed(_p(x), T, C, _p(qt), _p(s), _stream(x.device)))
+    return qt, s
+
+
+def weight_128x128(w: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tensor | None = None,
+                   transposed: bool = False, qt: torch.Tensor | None = None):
+    """w[N,K] bf16 -> (q[N,K] uint8, s[N/128, K/128] fp32, qt[K,N] uint8 or None)."""
+    _require(w, "w", torch.bfloat16, 2)
+    N, K = w.shape
+    q = _out(q, (N, K), torch.uint8, w.device, "q")
+    s = _out(s, (N // 128, K // 128), torch.float32, w.device, "s")
+    if transposed or qt is not None:
+        qt = _out(qt, (K, N), torch.uint8, w.device, "qt")
+    _check("fp8q_weight_128x128",
+           lib().fp8q_weight_128x128(_p(w), N, K, _p(q), _p(s), _p(qt), _stream(w.device)))
+    return q, s, qt
+
+
+# ------------------------------------------------------------------------------------------ #
+# GEMMs
+# ------------------------------------------------------------------------------------------ #
+
+def gemm_blockscaled(mode: int, A: torch.Tensor, sA: torch.Tensor, B: torch.Tensor,
+                     sB: torch.Tensor, out: torch.Tensor | None = None):
+    """Block-scaled FP8 GEMM.  FPROP: B = W[N,K]; DGRAD: B = W[K,N]; WGRAD: B = X^T[N,K].
+    Returns D[M,N] (bf16, or fp32 for WGRAD)."""
+    _require(A, "A", torch.uint8, 2)
+    _require(B, "B", torch.uint8, 2)
+    _require(sA, "sA", torch.float32, 2)
+    _require(sB, "sB", torch.float32, 2)
+    M, K = A.shape
+    N = B.shape[1] if mode == DGRAD else B.shape[0]
+    Kb = B.shape[0] if mode == DGRAD else B.shape[1]
+    if Kb != K:
+        raise ValueError(f"inner dimensions differ: A has K={K}, B has {Kb}")
+    dtype = torch.float32 if mode == WGRAD else torch.bfloat16
+    out = _out(out, (M, N), dtype, A.device, "out")
+    _check("fp8_gemm_blockscaled",
+           lib().fp8_gemm_blockscaled(int(mode), _p(A), _p(sA), _p(B), _p(sB), _p(out), M, N, K,
+                                      None, 0, _stream(A.device)))
+    return out
+
+
+def grouped_gemm_blockscaled(A: torch.Tensor, sA: torch.Tensor, B: torch.Tensor,
+                             sB: torch.Tensor, offsets: torch.Tensor,
+                             out: torch.Tensor | None = None):
+    """Grouped Fprop: A[Mtot,K], sA[K/128,Mtot], B[E,N,K], sB[E,N/128,K/128],
+    offsets int32[E+1] on the device.  Returns D[Mtot,N] bf16."""
+    _require(A, "A", torch.uint8, 2)
+    _require(B, "B", torch.uint8, 3)
+    _require(sA, "sA", torch.float32, 2)
+    _require(sB, "sB", torch.float32, 3)
+    _require(offsets, "offsets", torch.int32, 1)
+    Mtot, K = A.shape
+    E, N, Kb = B.shape
+    if Kb != K:
+        raise ValueError("inner dimensions differ")
+    if offsets.numel() != E + 1:
+        raise ValueError("offsets must have E+1 entries")
+    out = _out(out, (Mtot, N), torch.bfloat16, A.device, "out")
+    _check("fp8_grouped_gemm_blockscaled",
+           lib().fp8_grouped_gemm_blockscaled(_p(A), _p(sA), _p(B), _p(sB), _p(offsets), E, Mtot,
+                                              N, K, _p(out), _stream(A.device)))
+    return out
+
+
+def device_status(device: torch.device | None = None) -> int:
+    """Synchronise the current stream and return (and clear) the device status word."""
+    device = device or torch.device("cuda", torch.cuda.current_device())
+    v = ctypes.c_int(-1)
+    _check("fp8q_device_status", lib().fp8q_device_status(_stream(device), ctypes.byref(v)))
+    return int(v.value)
+
+
+def selftest_wait_timeout(limit_ns: int = 10_000_000, device: torch.device | None = None) -> None:
+    """Launch the timeout self-test kernel (see include/fp8q.h)."""
+    device = device or torch.device("cuda", torch.cuda.current_device())
+    _check("fp8q_selftest_wait_timeout",
+           lib().fp8q_selftest_wait_timeout(int(limit_ns), _stream(device)))

@@ -1,0 +1,175 @@
+/*
+ * fp8q.h -- C ABI of libfp8q.so: fine-grained FP8 (E4M3) quantisation and the block-scaled
+ * FP8 GEMM of DeepSeek-V3's linear layers, hand-written for B200 (sm_100a).
+ *
+ * Passages these operations follow (pages on the DeepSeek-V3 Technical Report, arXiv
+ * 2412.19437):
+ *   [SUMMARY] "DeepSeek-V3 Technical Report" summary page (xyznot.com): Key ideas, FP8
+ *             mixed-precision bullet -- E4M3 for all tensors, 1x128 tile-wise activation and
+ *             128x128 block-wise weight scaling, accumulation copied to FP32 CUDA-core registers
+ *             every N_c = 128 elements; Questions, the answer on FP8 training without
+ *             divergence -- the same, restated.
+ *   [REPOST]  DeepSeek-V3 report repost (why-be.co.kr board post): paragraph 1 -- 128 elements
+ *             (4 WGMMAs) is the promotion interval; paragraph 2 and Figure 6 -- Fprop, Dgrad
+ *             and Wgrad all run in FP8; paragraph 3 -- master weights and gradients stay in
+ *             FP32; paragraph 4 -- per-group scaling factors along the GEMM's inner dimension,
+ *             dequantised during the increased-precision accumulation (Figure 7(b)).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Every pointer argument is a DEVICE pointer owned by the caller (for example a PyTorch
+ *   tensor's data_ptr()).  The library never allocates, frees or retains caller memory.
+ * - Every tensor is dense row-major with no padding; bf16 tensors are passed as uint16_t bit
+ *   patterns; E4M3 codes as uint8_t (OCP E4M3FN: bias 7, largest finite 448 = 0x7E).
+ * - Every data pointer must be 16-byte aligned (FP8Q_ERR_ALIGN otherwise).
+ * - Work is enqueued on `stream` (NULL = the legacy default stream) and is complete when the
+ *   stream reaches it.  No call synchronises, except fp8q_device_status.
+ * - The status returned covers the host-side checks and the launch only.  Errors found on the
+ *   device (a malformed offsets array, a pipeline wait that timed out) are latched in a device
+ *   status word that fp8q_device_status reads and clears.
+ * - A call with an empty problem (M == 0, T == 0, ...) returns FP8Q_OK and launches nothing.
+ * - Scale layout: the per-row scales of a [rows, K] operand quantised in groups of 128 along K
+ *   are stored group-major, s[K/128][rows], so one 128-row tile's scales for one K group are
+ *   one contiguous 512-byte run.
+ * - Quantisation of a group g: a = max(max|x| over g, 2^-100); s = a / 448 (stored: the
+ *   dequantisation multiplier); q = E4M3(x * (448 / a)) rounded to nearest even with
+ *   saturation.  The divisions and the multiply are IEEE binary32, round to nearest.  Codes and
+ *   scales are bit-exact functions of the input.
+ */
+#ifndef FP8Q_H
+#define FP8Q_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FP8Q_API __attribute__((visibility("default")))
+#else
+#define FP8Q_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL selects the legacy default stream. */
+typedef struct CUstream_st* fp8q_stream_t;
+
+/* Return codes. */
+enum {
+    FP8Q_OK = 0,
+    FP8Q_ERR_ARG = 1,          /* null pointer where data is required, negative size, bad mode */
+    FP8Q_ERR_SHAPE = 2,        /* a dimension that a 128-group spans is not a multiple of 128 */
+    FP8Q_ERR_ALIGN = 3,        /* a data pointer is not 16-byte aligned */
+    FP8Q_ERR_CUDA = 4,         /* a CUDA runtime or driver call failed (no device, launch error) */
+    FP8Q_ERR_UNSUPPORTED = 5,  /* a size beyond what this build supports (see each call) */
+    FP8Q_ERR_DEVICE = 6        /* reported by fp8q_device_status: an error latched on the device */
+};
+
+/* Device status word values (what fp8q_device_status writes to *out). */
+enum {
+    FP8Q_DEV_OK = 0,
+    FP8Q_DEV_TIMEOUT = 1,      /* a bounded pipeline wait expired; the kernel exited early */
+    FP8Q_DEV_BAD_OFFSETS = 2   /* grouped GEMM: offsets not 0-based / nondecreasing / ending at Mtot */
+};
+
+/* GEMM modes (the three GEMMs of a linear layer, [REPOST] paragraph 2, Figure 6). */
+enum {
+    FP8Q_FPROP = 0,            /* Y  = X  W^T : D bf16 */
+    FP8Q_DGRAD = 1,            /* dX = dY W   : D bf16 */
+    FP8Q_WGRAD = 2             /* dW = dY^T X : D fp32 */
+};
+
+/* Human-readable name of a return code (static storage; never NULL). */
+FP8Q_API const char* fp8q_status_string(int status);
+
+/* ABI version of this header (incremented on incompatible change). */
+FP8Q_API int fp8q_abi_version(void);
+
+/*
+ * 1x128 tile-wise activation quantisation ([SUMMARY] Key ideas, FP8 bullet).
+ *   x : [M, K] bf16            q : [M, K] E4M3 codes         s : [K/128, M] fp32 scales
+ * Group = one row, 128 consecutive columns.  K % 128 == 0 (FP8Q_ERR_SHAPE otherwise); any
+ * M >= 0.  x is not modified; q and s are fully overwritten.
+ */
+FP8Q_API int fp8q_act_1x128(const uint16_t* x, int64_t M, int64_t K, uint8_t* q, float* s,
+                   fp8q_stream_t stream);
+
+/*
+ * 128x1 token-direction quantisation with transposed output, the operand form of Wgrad, whose
+ * inner (scaled) dimension is the token dimension ([REPOST] paragraphs 2 and 4).
+ *   x : [T, C] bf16            qt : [C, T] E4M3 codes        s : [T/128, C] fp32 scales
+ * Group = one channel c, 128 consecutive tokens.  T % 128 == 0 and C % 64 == 0
+ * (FP8Q_ERR_SHAPE otherwise).
+ */
+FP8Q_API int fp8q_act_128x1_transposed(const uint16_t* x, int64_t T, int64_t C, uint8_t* qt, float* s,
+                              fp8q_stream_t stream);
+
+/*
+ * 128x128 block-wise weight quantisation ([SUMMARY] Key ideas, FP8 bullet).
+ *   w : [N, K] bf16            q : [N, K] E4M3 codes         s : [N/128, K/128] fp32 scales
+ *   qt_or_null : NULL, or [K, N] receiving the same codes transposed.
+ * N % 128 == 0 and K % 128 == 0 (FP8Q_ERR_SHAPE otherwise).
+ */
+FP8Q_API int fp8q_weight_128x128(const uint16_t* w, int64_t N, int64_t K, uint8_t* q, float* s,
+                        uint8_t* qt_or_null, fp8q_stream_t stream);
+
+/*
+ * Block-scaled FP8 GEMM with FP32 promotion every 128 K ([REPOST] paragraphs 1 and 4;
+ * [SUMMARY] FP8 bullet):  D[m, n] = sum_kb sum_{k in kb} A^(m, k) B^(k, n), where each 128-wide
+ * K group's tensor-core partial sum is multiplied by its two scales and added into an FP32
+ * accumulator.
+ *
+ *   A  : [M, K] E4M3 codes, sA : [K/128, M] (1x128 or 128x1-transposed scales).
+ *   mode FP8Q_FPROP: B = W [N, K] codes, sB = [N/128, K/128] block scales; D = bf16 [M, N].
+ *   mode FP8Q_DGRAD: B = W [K, N] codes -- the forward weight [out = K, in = N], used
+ *                    transposed, no requantisation; sB = [K/128, N/128]; D = bf16 [M, N].
+ *   mode FP8Q_WGRAD: B = X^T [N, K] codes (128x1 along K = tokens), sB = [K/128, N];
+ *                    D = fp32 [M, N].
+ * Requirements: K % 128 == 0, N % 128 == 0 (FP8Q_ERR_SHAPE); M >= 0 (any M, the last row tile
+ * is masked); K/128 < 2^24.  D is fully overwritten (no accumulation into D).
+ * workspace / ws_bytes: reserved for split-K schedules; pass NULL / 0.  fp8q_gemm_workspace_size
+ * reports the bytes a call needs (currently always 0).
+ */
+FP8Q_API int fp8_gemm_blockscaled(int mode, const uint8_t* A, const float* sA, const uint8_t* B,
+                         const float* sB, void* D, int64_t M, int64_t N, int64_t K,
+                         void* workspace, size_t ws_bytes, fp8q_stream_t stream);
+
+FP8Q_API size_t fp8q_gemm_workspace_size(int mode, int64_t M, int64_t N, int64_t K);
+
+/*
+ * Grouped (MoE expert) block-scaled FP8 Fprop over ragged row groups: the rows of A are sorted
+ * by expert and rows offsets[e] .. offsets[e+1]-1 multiply expert e's weight.
+ *   A  : [Mtot, K] codes, sA : [K/128, Mtot]
+ *   B  : [E, N, K] codes, sB : [E, N/128, K/128]
+ *   offsets : DEVICE int32 [E + 1], offsets[0] = 0, nondecreasing, offsets[E] = Mtot.  Empty
+ *             experts are allowed.  A malformed array is detected on the device: nothing is
+ *             written and FP8Q_DEV_BAD_OFFSETS is latched for fp8q_device_status.
+ *   D  : [Mtot, N] bf16.
+ * Requirements: K % 128 == 0, N % 128 == 0, 1 <= E <= 1024, Mtot < 2^31.
+ */
+FP8Q_API int fp8_grouped_gemm_blockscaled(const uint8_t* A, const float* sA, const uint8_t* B,
+                                 const float* sB, const int32_t* offsets, int32_t E,
+                                 int64_t Mtot, int64_t N, int64_t K, uint16_t* D,
+                                 fp8q_stream_t stream);
+
+/*
+ * Synchronise `stream`, then read and clear the device status word of the current device.
+ * *out receives FP8Q_DEV_OK or the first error latched since the last call.  Returns FP8Q_OK,
+ * FP8Q_ERR_ARG (out == NULL) or FP8Q_ERR_CUDA.
+ */
+FP8Q_API int fp8q_device_status(fp8q_stream_t stream, int* out);
+
+/*
+ * Self-test of the device-side error path (no counterpart on the pages): launches one CTA that
+ * waits on a barrier nothing ever completes, with the same bounded wait the GEMM pipeline uses
+ * but a limit of `limit_ns` (1 .. 2e9).  The wait expires, FP8Q_DEV_TIMEOUT is latched and the
+ * kernel returns; the context stays usable.  Returns FP8Q_ERR_ARG for a limit out of range.
+ */
+FP8Q_API int fp8q_selftest_wait_timeout(uint64_t limit_ns, fp8q_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8Q_H */

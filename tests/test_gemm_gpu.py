@@ -1,0 +1,244 @@
+"""GPU block-scaled FP8 GEMM vs the CPU oracle (Fprop, Dgrad, Wgrad).
+
+* Exact cases: dyadic operands whose groups have power-of-two scales and whose products
+  cancel nowhere but sum to small integers times powers of two; the exact result is
+  representable in the output type, so any correct kernel returns it bit for bit.
+* Tolerance cases: realistic operands (oracle-quantised synthetic activations, weights and
+  gradients) over several tiles with ragged row counts, both tile widths, full outputs.
+* Full-size cases, the shapes the benchmark times: sampled rows, columns and entries.
+The quantised operands are always produced by the oracle on the host, never by the GPU.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fp8_fine_grained_fp8q_b200 import ops, synth
+from tests._util import check_gemm, f32_dev, host, linear_layer_inputs, u8_dev
+
+pytestmark = pytest.mark.gpu
+
+FPROP, DGRAD, WGRAD = ops.FPROP, ops.DGRAD, ops.WGRAD
+
+
+def run_gemm(mode, A, sA, B, sB, bn=None, monkeypatch=None):
+    if bn is not None:
+        monkeypatch.setenv("FP8Q_GEMM_BN", str(bn))
+    M = A.shape[0]
+    N = B.shape[1] if mode == DGRAD else B.shape[0]
+    dtype = torch.float32 if mode == WGRAD else torch.bfloat16
+    out = torch.full((M, N), float("nan"), dtype=dtype, device="cuda")
+    ops.gemm_blockscaled(mode, u8_dev(A), f32_dev(sA), u8_dev(B), f32_dev(sB), out=out)
+    assert ops.device_status() == ops.DEV_OK
+    return host(out)
+
+
+# ------------------------------------------------------------------------------------------ #
+# Exact dyadic cases
+# ------------------------------------------------------------------------------------------ #
+
+def _ternary(g, shape, density=0.25):
+    v = g.integers(-1, 2, size=shape).astype(np.float32)
+    return v * (g.random(shape) < density)
+
+
+def _bits(x):
+    return synth.f32_to_bf16_bits(x)
+
+
+def exact_fprop(M, N, K, seed):
+    g = np.random.Generator(np.random.PCG64(seed))
+    jx = g.integers(-4, 5, size=M)
+    jw = g.integers(-4, 5, size=N // 128)
+    X = _ternary(g, (M, K))
+    W = _ternary(g, (N, K))
+    X[:, 1::128] = 0.0
+    W[:, 0::128] = 0.0
+    X[:, 0::128] = 448.0 * np.where(g.random((M, K // 128)) < 0.5, -1, 1)
+    for nb in range(N // 128):
+        W[nb * 128, 1::128] = 448.0
+    X *= np.exp2(jx)[:, None].astype(np.float32)
+    W *= np.exp2(np.repeat(jw, 128))[:, None].astype(np.float32)
+    exact = X.astype(np.float64) @ W.astype(np.float64).T
+    return X, W, exact
+
+
+@pytest.mark.parametrize("bn", [128, 256])
+@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (200, 512, 384), (1, 256, 128), (384, 256, 1024)])
+def test_exact_fprop(M, N, K, bn, monkeypatch):
+    X, W, exact = exact_fprop(M, N, K, seed=M + N + K)
+    # Representable in bf16: integers of magnitude <= 256 times a power of two.
+    ints = exact / np.exp2(np.floor(np.log2(np.maximum(np.abs(exact), 1e-300))) - 7)
+    assert np.all((exact == 0) | (np.abs(ints - np.round(ints)) == 0))
+    xq, xs = oracle.quant_1x128(_bits(X))
+    wq, ws, _ = oracle.quant_128x128(_bits(W))
+    ref, _ = oracle.gemm(FPROP, xq, xs, wq, ws)
+    assert np.array_equal(ref, exact)
+    got = run_gemm(FPROP, xq, xs, wq, ws, bn, monkeypatch)
+    assert np.array_equal(got, exact)
+
+
+@pytest.mark.parametrize("bn", [128, 256])
+@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (260, 512, 384)])
+def test_exact_dgrad(M, N, K, bn, monkeypatch):
+    # dX[M,N] = dY[M,K] W[K,N]; W is the forward weight [out=K, in=N].
+    g = np.random.Generator(np.random.PCG64(M * N + K))
+    jy = g.integers(-4, 5, size=M)
+    jw = g.integers(-4, 5, size=N // 128)
+    dY = _ternary(g, (M, K))
+    W = _ternary(g, (K, N))
+    dY[:, 1::128] = 0.0
+    W[0::128, :] = 0.0
+    dY[:, 0::128] = 448.0
+    for nb in range(N // 128):
+        W[1::128, nb * 128] = -448.0
+    dY *= np.exp2(jy)[:, None].astype(np.float32)
+    W *= np.exp2(np.repeat(jw, 128))[None, :].astype(np.float32)
+    exact = dY.astype(np.float64) @ W.astype(np.float64)
+    gq, gs = oracle.quant_1x128(_bits(dY))
+    wq, ws, _ = oracle.quant_128x128(_bits(W))
+    got = run_gemm(DGRAD, gq, gs, wq, ws, bn, monkeypatch)
+    assert np.array_equal(got, exact)
+
+
+@pytest.mark.parametrize("bn", [128, 256])
+@pytest.mark.parametrize("T,Cout,Cin", [(128, 128, 256), (512, 384, 512)])
+def test_exact_wgrad(T, Cout, Cin, bn, monkeypatch):
+    # dW[Cout,Cin] = dY[T,Cout]^T X[T,Cin]; FP32 output, so larger sums stay exact.
+    g = np.random.Generator(np.random.PCG64(T + Cout * Cin))
+    jy = g.integers(-4, 5, size=Cout)
+    jx = g.integers(-4, 5, size=Cin)
+    dY = g.integers(-8, 9, size=(T, Cout)).astype(np.float32)
+    X = g.integers(-8, 9, size=(T, Cin)).astype(np.float32)
+    dY[1::128, :] = 0.0
+    X[0::128, :] = 0.0
+    dY[0::128, :] = 448.0
+    X[1::128, :] = -448.0
+    dY *= np.exp2(jy)[None, :].astype(np.float32)
+    X *= np.exp2(jx)[None, :].astype(np.float32)
+    exact = dY.astype(np.float64).T @ X.astype(np.float64)
+    gq, gs = oracle.quant_128x1_t(_bits(dY))
+    xq, xs = oracle.quant_128x1_t(_bits(X))
+    got = run_gemm(WGRAD, gq, gs, xq, xs, bn, monkeypatch)
+    assert np.array_equal(got, exact)
+
+
+# ------------------------------------------------------------------------------------------ #
+# Tolerance cases, full outputs
+# ------------------------------------------------------------------------------------------ #
+
+def test_tiny_fprop_workload():
+    d = synth.tiny_fprop()
+    xq, xs = oracle.quant_1x128(d["X"])
+    wq, ws, _ = oracle.quant_128x128(d["W"])
+    ref, S = oracle.gemm(FPROP, xq, xs, wq, ws)
+    got = run_gemm(FPROP, xq, xs, wq, ws)
+    check_gemm(got, ref, S, "tiny fprop 256x512x512")
+
+
+@pytest.mark.parametrize("bn", [128, 256])
+@pytest.mark.parametrize("M,N,K", [(200, 256, 384), (517, 512, 1024), (1, 256, 256)])
+def test_fprop_ragged(M, N, K, bn, monkeypatch):
+    X = synth.activations_channel_outliers(M, K, seed=M + K)
+    W = synth.weights(N, K, seed=N + K + 1)
+    xq, xs = oracle.quant_1x128(X)
+    wq, ws, _ = oracle.quant_128x128(W)
+    ref, S = oracle.gemm(FPROP, xq, xs, wq, ws)
+    check_gemm(run_gemm(FPROP, xq, xs, wq, ws, bn, monkeypatch), ref, S, f"fprop {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("bn", [128, 256])
+@pytest.mark.parametrize("M,N,K", [(256, 512, 256), (333, 768, 640)])
+def test_dgrad_ragged(M, N, K, bn, monkeypatch):
+    dY = synth.output_grad(M, K, seed=M + K)
+    W = synth.weights(K, N, seed=N + K + 2)
+    gq, gs = oracle.quant_1x128(dY)
+    wq, ws, _ = oracle.quant_128x128(W)
+    ref, S = oracle.gemm(DGRAD, gq, gs, wq, ws)
+    check_gemm(run_gemm(DGRAD, gq, gs, wq, ws, bn, monkeypatch), ref, S, f"dgrad {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("bn", [128, 256])
+@pytest.mark.parametrize("T,Cout,Cin", [(512, 256, 512), (384, 384, 768)])
+def test_wgrad(T, Cout, Cin, bn, monkeypatch):
+    dY = synth.output_grad(T, Cout, seed=T + Cout)
+    X = synth.activations_channel_outliers(T, Cin, seed=T + Cin + 3)
+    gq, gs = oracle.quant_128x1_t(dY)
+    xq, xs = oracle.quant_128x1_t(X)
+    ref, S = oracle.gemm(WGRAD, gq, gs, xq, xs)
+    check_gemm(run_gemm(WGRAD, gq, gs, xq, xs, bn, monkeypatch), ref, S, f"wgrad {T}x{Cout}x{Cin}")
+
+
+def test_empty_rows_is_a_no_op():
+    A = torch.zeros((0, 256), dtype=torch.uint8, device="cuda")
+    sA = torch.zeros((2, 0), dtype=torch.float32, device="cuda")
+    B = torch.zeros((128, 256), dtype=torch.uint8, device="cuda")
+    sB = torch.ones((1, 2), dtype=torch.float32, device="cuda")
+    out = ops.gemm_blockscaled(FPROP, A, sA, B, sB)
+    assert out.shape == (0, 128)
+
+
+# ------------------------------------------------------------------------------------------ #
+# Full-size shapes (sampled against the oracle)
+# ------------------------------------------------------------------------------------------ #
+
+_q = {}
+
+
+def quantised_layer():
+    if not _q:
+        d = linear_layer_inputs()
+        _q["X"] = oracle.quant_1x128(d["X"])
+        _q["dY"] = oracle.quant_1x128(d["dY"])
+        _q["W"] = oracle.quant_128x128(d["W"])[:2]
+        _q["Xt"] = oracle.quant_128x1_t(d["X"])
+        _q["dYt"] = oracle.quant_128x1_t(d["dY"])
+    return _q
+
+
+def sampled_check(mode, A, sA, B, sB, got, what, seed=0):
+    M, N = got.shape
+    g = np.random.Generator(np.random.PCG64(seed))
+    rows = np.unique([0, 127, 128, M // 2 + 3, M - 1])
+    cols = np.unique([0, 127, 128, N // 2 + 5, N - 1])
+    ms = [np.repeat(rows, N), np.tile(np.arange(N), rows.size)]
+    ns_ = [np.tile(np.arange(M), cols.size), np.repeat(cols, M)]
+    rm, rn = g.integers(0, M, 4096), g.integers(0, N, 4096)
+    mm = np.concatenate([ms[0], ns_[0], rm])
+    nn = np.concatenate([ms[1], ns_[1], rn])
+    ref, S = oracle.gemm_entries(mode, A, sA, B, sB, mm, nn)
+    assert np.all(np.isfinite(got)), f"{what}: unwritten or non-finite outputs"
+    return check_gemm(got[mm, nn], ref, S, what)
+
+
+def test_full_fprop_ffn_up():
+    q = quantised_layer()
+    (xq, xs), (wq, ws) = q["X"], q["W"]
+    got = run_gemm(FPROP, xq, xs, wq, ws)
+    sampled_check(FPROP, xq, xs, wq, ws, got, "fprop 4096x2048x7168")
+
+
+def test_full_dgrad():
+    q = quantised_layer()
+    (gq, gs), (wq, ws) = q["dY"], q["W"]
+    got = run_gemm(DGRAD, gq, gs, wq, ws)
+    assert got.shape == (4096, 7168)
+    sampled_check(DGRAD, gq, gs, wq, ws, got, "dgrad 4096x7168x2048")
+
+
+def test_full_wgrad():
+    q = quantised_layer()
+    (gq, gs), (xq, xs) = q["dYt"], q["Xt"]
+    got = run_gemm(WGRAD, gq, gs, xq, xs)
+    assert got.shape == (2048, 7168)
+    sampled_check(WGRAD, gq, gs, xq, xs, got, "wgrad 2048x7168x4096")
+
+
+@pytest.mark.parametrize("N", [1536, 512])
+def test_full_fprop_mla(N):
+    q = quantised_layer()
+    xq, xs = q["X"]
+    W = synth.weights(N, 7168, seed=synth.SEED_BASE + 3 + N)
+    wq, ws, _ = oracle.quant_128x128(W)
+    got = run_gemm(FPROP, xq, xs, wq, ws)
+    sampled_check(FPROP, xq, xs, wq, ws, got, f"fprop MLA 4096x{N}x7168")
