@@ -137,18 +137,16 @@ int launch_gemm(const uint8_t* A, const float* sA, const uint8_t* B, const float
     return launch_status();
 }
 
-// Tile width: 256 unless 128-wide tiles finish in fewer waves of persistent CTAs.
+// Tile width: 256 whenever N allows it (measured faster on every linear-layer and MLA shape: it
+// halves the B-tile traffic per MMA and gives the promotion warps twice the MMA time per group);
+// FP8Q_GEMM_BN=128 forces the narrow tile (tests and tuning).
 int choose_bn(int64_t M, int64_t N, int extra_m_tiles)
 {
+    (void)M;
+    (void)extra_m_tiles;
     const char* env = getenv("FP8Q_GEMM_BN");
-    if (env && (N % 256 == 0) && atoi(env) == 256) return 256;
     if (env && atoi(env) == 128) return 128;
-    if (N % 256 != 0) return 128;
-    const int sms = sm_count() > 0 ? sm_count() : 148;
-    const int64_t mt = (M + 127) / 128 + extra_m_tiles;
-    const int64_t w256 = (mt * (N / 256) + sms - 1) / sms;   // waves of 256-wide tiles (cost 2 each)
-    const int64_t w128 = (mt * (N / 128) + sms - 1) / sms;   // waves of 128-wide tiles (cost 1 each)
-    return (2 * w256 <= w128) ? 256 : 128;
+    return (N % 256 == 0) ? 256 : 128;
 }
 
 template <int MODE>

@@ -293,7 +293,11 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
         const int rit = quad * 32 + lane;     // row within the tile
         int tb = 0, ss = 0;
         uint32_t tph = 0, sph = 0;
-        float acc[S::kHalf];
+        // Columns per TMEM load: 16 at BN = 256 (two chunks in flight still fit beside the 128
+        // accumulators), 32 at BN = 128.
+        constexpr int kCW = 16;
+        constexpr int kChunks = S::kHalf / kCW;
+        float2 acc[S::kHalf / 2];
         for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
             const TileInfo ti = decode_tile<GROUPED>(t, nb_tiles, BN, args, g_off, g_pre);
             const int row = ti.row0 + rit;
@@ -310,7 +314,7 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                 sb_step = (size_t)(args.N >> 7);
             }
 #pragma unroll
-            for (int i = 0; i < S::kHalf; ++i) acc[i] = 0.0f;
+            for (int i = 0; i < S::kHalf / 2; ++i) acc[i] = make_float2(0.0f, 0.0f);
             float sa_next = in_a ? __ldg(sa_ptr) : 0.0f;
             float sb_next = (MODE != kModeWgrad) ? __ldg(sb_ptr) : 1.0f;
             bool ok = true;
@@ -321,41 +325,64 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                     if (MODE != kModeWgrad) sb_next = __ldg(sb_ptr + (size_t)(kb + 1) * sb_step);
                 }
                 if (!warp_wait(tfull_bar(tb), tph, abort_flag)) { ok = false; break; }
+                if (MODE == kModeWgrad) {
+                    if (!warp_wait(sfull_bar(ss), sph, abort_flag)) { ok = false; break; }
+                }
                 tc_fence_after();
                 const uint32_t taddr = tmem_base + lane_base + (uint32_t)(tb * BN + half * S::kHalf);
-                if (MODE != kModeWgrad) {
-                    const float c = sa * sbv;
+                const float* cs = col_scales + ss * BN + half * S::kHalf;
+                const float2 c2 = make_float2(sa * sbv, sa * sbv);
+                const float2 sa2 = make_float2(sa, sa);
+                // Two register chunks: the TMEM load of chunk ch+1 is in flight while chunk ch is
+                // folded into the accumulators.  The buffer is released as soon as its last
+                // chunk has landed in registers, before that chunk's arithmetic.
+                uint32_t ra[kCW], rb[kCW];
+                tmem_ld_async(taddr, ra);
+                tmem_wait_ld(ra);
+                const auto fold = [&](uint32_t (&cur)[kCW], int ch) {
+                    if (MODE != kModeWgrad) {
 #pragma unroll
-                    for (int ch = 0; ch < S::kHalf / 32; ++ch) {
-                        float v[32];
-                        tmem_ld32(taddr + ch * 32, v);
+                        for (int j = 0; j < kCW; j += 2) {
+                            const float2 v = make_float2(__uint_as_float(cur[j]), __uint_as_float(cur[j + 1]));
+                            acc[(ch * kCW + j) / 2] = __ffma2_rn(v, c2, acc[(ch * kCW + j) / 2]);
+                        }
+                    } else {
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) acc[ch * 32 + j] = fmaf(v[j], c, acc[ch * 32 + j]);
-                    }
-                } else {
-                    if (!warp_wait(sfull_bar(ss), sph, abort_flag)) { ok = false; break; }
-                    const float* cs = col_scales + ss * BN + half * S::kHalf;
-#pragma unroll
-                    for (int ch = 0; ch < S::kHalf / 32; ++ch) {
-                        float v[32];
-                        tmem_ld32(taddr + ch * 32, v);
-#pragma unroll
-                        for (int j = 0; j < 32; j += 4) {
-                            const float4 c4 = *reinterpret_cast<const float4*>(cs + ch * 32 + j);
-                            acc[ch * 32 + j + 0] = fmaf(v[j + 0], sa * c4.x, acc[ch * 32 + j + 0]);
-                            acc[ch * 32 + j + 1] = fmaf(v[j + 1], sa * c4.y, acc[ch * 32 + j + 1]);
-                            acc[ch * 32 + j + 2] = fmaf(v[j + 2], sa * c4.z, acc[ch * 32 + j + 2]);
-                            acc[ch * 32 + j + 3] = fmaf(v[j + 3], sa * c4.w, acc[ch * 32 + j + 3]);
+                        for (int j = 0; j < kCW; j += 4) {
+                            const float4 c4 = *reinterpret_cast<const float4*>(cs + ch * kCW + j);
+                            const float2 s01 = __fmul2_rn(sa2, make_float2(c4.x, c4.y));
+                            const float2 s23 = __fmul2_rn(sa2, make_float2(c4.z, c4.w));
+                            const float2 v01 = make_float2(__uint_as_float(cur[j]), __uint_as_float(cur[j + 1]));
+                            const float2 v23 = make_float2(__uint_as_float(cur[j + 2]), __uint_as_float(cur[j + 3]));
+                            acc[(ch * kCW + j) / 2] = __ffma2_rn(v01, s01, acc[(ch * kCW + j) / 2]);
+                            acc[(ch * kCW + j) / 2 + 1] = __ffma2_rn(v23, s23, acc[(ch * kCW + j) / 2 + 1]);
                         }
                     }
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(tempty_bar(tb));
-                    if (MODE == kModeWgrad) mbar_arrive(sempty_bar(ss));
+                };
+                const auto release = [&]() {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(tempty_bar(tb));
+                };
+#pragma unroll
+                for (int ch = 0; ch < kChunks; ++ch) {
+                    if (ch + 1 < kChunks) {
+                        if (ch & 1) tmem_ld_async(taddr + (ch + 1) * kCW, ra);
+                        else tmem_ld_async(taddr + (ch + 1) * kCW, rb);
+                    } else {
+                        release();
+                    }
+                    if (ch & 1) fold(rb, ch); else fold(ra, ch);
+                    if (ch + 1 < kChunks) {
+                        if (ch & 1) tmem_wait_ld(ra); else tmem_wait_ld(rb);
+                    }
                 }
                 if (MODE == kModeWgrad) {
+                    // The column scales were read with ordinary loads; the next bulk copy into this
+                    // slot is an async-proxy write, so fence the proxies before releasing it.
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(sempty_bar(ss));
                     if (++ss == S::kScaleStages) { ss = 0; sph ^= 1u; }
                 }
                 if (++tb == 2) { tb = 0; tph ^= 1u; }
@@ -366,18 +393,19 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                 if (MODE == kModeWgrad) {
                     float* drow = reinterpret_cast<float*>(args.D) + (size_t)row * args.N + ncol0;
 #pragma unroll
-                    for (int j = 0; j < S::kHalf; j += 4)
-                        *reinterpret_cast<float4*>(drow + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+                    for (int j = 0; j < S::kHalf / 2; j += 2)
+                        *reinterpret_cast<float4*>(drow + 2 * j) =
+                            make_float4(acc[j].x, acc[j].y, acc[j + 1].x, acc[j + 1].y);
                 } else {
                     uint16_t* drow = reinterpret_cast<uint16_t*>(args.D) + (size_t)row * args.N + ncol0;
 #pragma unroll
-                    for (int j = 0; j < S::kHalf; j += 8) {
+                    for (int j = 0; j < S::kHalf / 2; j += 4) {
                         uint4 o;
-                        o.x = pack_bf16x2(acc[j + 0], acc[j + 1]);
-                        o.y = pack_bf16x2(acc[j + 2], acc[j + 3]);
-                        o.z = pack_bf16x2(acc[j + 4], acc[j + 5]);
-                        o.w = pack_bf16x2(acc[j + 6], acc[j + 7]);
-                        *reinterpret_cast<uint4*>(drow + j) = o;
+                        o.x = pack_bf16x2(acc[j + 0].x, acc[j + 0].y);
+                        o.y = pack_bf16x2(acc[j + 1].x, acc[j + 1].y);
+                        o.z = pack_bf16x2(acc[j + 2].x, acc[j + 2].y);
+                        o.w = pack_bf16x2(acc[j + 3].x, acc[j + 3].y);
+                        *reinterpret_cast<uint4*>(drow + 2 * j) = o;
                     }
                 }
             }
