@@ -7,7 +7,9 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
+#include <random>
 
 #include "fp8q.h"
 #include "gemm.cuh"
@@ -102,9 +104,43 @@ int prepare_kernel()
     return ready[dev] == 1 ? FP8Q_OK : FP8Q_ERR_UNSUPPORTED;
 }
 
+// Workspace of the stream-K schedule for `ctas` persistent CTAs of BN-wide tiles: one FP32
+// 128 x BN partial slot per CTA, then one 64-bit ready flag per CTA (256-byte aligned).
+size_t sk_slot_bytes(int bn) { return (size_t)128 * bn * sizeof(float); }
+size_t sk_workspace_bytes(int ctas, int bn)
+{
+    return (size_t)ctas * sk_slot_bytes(bn) + (((size_t)ctas * sizeof(uint64_t) + 255) & ~(size_t)255);
+}
+
+// Launch stamps: a flag holds the stamp of the launch that published it, so flags are never
+// reset.  The high half is random per process (stale workspace contents cannot match by
+// accident), the low half counts launches.
+unsigned long long next_stamp()
+{
+    static std::atomic<unsigned long long> counter{0};
+    static const unsigned long long salt = [] {
+        std::random_device rd;
+        unsigned long long v = ((unsigned long long)rd() << 32) ^ (unsigned long long)rd();
+        return v | 1ull;
+    }();
+    return (salt & 0xFFFFFFFF00000000ull) | ((++counter) & 0xFFFFFFFFull) | 1ull << 31;
+}
+
+// Stream-K pays off when the tiles do not fill whole waves of the persistent grid.
+// FP8Q_GEMM_SCHED=dp / sk forces the data-parallel / stream-K schedule.
+bool want_streamk(int64_t tiles, int ctas, int kb)
+{
+    const char* env = getenv("FP8Q_GEMM_SCHED");
+    if (env && strcmp(env, "dp") == 0) return false;
+    if (kb < 2) return false;
+    if (env && strcmp(env, "sk") == 0) return true;
+    return tiles % ctas != 0;
+}
+
 template <int MODE, int BN, bool GROUPED>
 int launch_gemm(const uint8_t* A, const float* sA, const uint8_t* B, const float* sB, void* D,
-                const int32_t* offsets, int E, int64_t M, int64_t N, int64_t K, cudaStream_t st)
+                const int32_t* offsets, int E, int64_t M, int64_t N, int64_t K, cudaStream_t st,
+                void* workspace = nullptr, size_t ws_bytes = 0)
 {
     using S = GemmShape<MODE, BN, GROUPED>;
     const int prep = prepare_kernel<MODE, BN, GROUPED>();
@@ -126,11 +162,42 @@ int launch_gemm(const uint8_t* A, const float* sA, const uint8_t* B, const float
     a.M = (int32_t)M;
     a.N = (int32_t)N;
     a.KB = (int32_t)(K / 128);
+    a.ws = nullptr;
+    a.flags = nullptr;
+    a.stamp = 0;
+    a.units = 0;
     const int sms = sm_count();
     if (sms <= 0) return FP8Q_ERR_CUDA;
     // Grouped: at most ceil(Mtot/128) + E row tiles (each group adds at most one partial tile).
     const int64_t m_tiles = GROUPED ? (M + 127) / 128 + E : (M + 127) / 128;
     const int64_t tiles = m_tiles * (N / BN);
+    const int64_t units = tiles * a.KB;
+    if (!GROUPED && workspace && want_streamk(tiles, sms, a.KB)) {
+        const int grid = (int)(units < sms ? units : sms);
+        if (ws_bytes >= sk_workspace_bytes(grid, BN) && (reinterpret_cast<uintptr_t>(workspace) & 255u) == 0) {
+            a.ws = static_cast<float*>(workspace);
+            a.flags = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(workspace) +
+                                                            (size_t)grid * sk_slot_bytes(BN));
+            a.stamp = next_stamp();
+            a.units = units;
+            // CTAs wait on each other's partials: launch them co-resident (cooperative launch).
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3((unsigned)grid);
+            cfg.blockDim = dim3(S::kThreads);
+            cfg.dynamicSmemBytes = S::kSmemBytes;
+            cfg.stream = st;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeCooperative;
+            attr[0].val.cooperative = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            if (cudaLaunchKernelEx(&cfg, gemm_blockscaled_kernel<MODE, BN, GROUPED>, ta, tb, a) != cudaSuccess) {
+                cudaGetLastError();
+                return FP8Q_ERR_CUDA;
+            }
+            return launch_status();
+        }
+    }
     const int grid = (int)(tiles < sms ? tiles : sms);
     if (grid <= 0) return FP8Q_OK;
     gemm_blockscaled_kernel<MODE, BN, GROUPED><<<grid, S::kThreads, S::kSmemBytes, st>>>(ta, tb, a);
@@ -151,11 +218,11 @@ int choose_bn(int64_t M, int64_t N, int extra_m_tiles)
 
 template <int MODE>
 int gemm_mode(const uint8_t* A, const float* sA, const uint8_t* B, const float* sB, void* D, int64_t M,
-              int64_t N, int64_t K, cudaStream_t st)
+              int64_t N, int64_t K, cudaStream_t st, void* ws, size_t ws_bytes)
 {
     if (choose_bn(M, N, 0) == 256)
-        return launch_gemm<MODE, 256, false>(A, sA, B, sB, D, nullptr, 1, M, N, K, st);
-    return launch_gemm<MODE, 128, false>(A, sA, B, sB, D, nullptr, 1, M, N, K, st);
+        return launch_gemm<MODE, 256, false>(A, sA, B, sB, D, nullptr, 1, M, N, K, st, ws, ws_bytes);
+    return launch_gemm<MODE, 128, false>(A, sA, B, sB, D, nullptr, 1, M, N, K, st, ws, ws_bytes);
 }
 
 // Waits on an mbarrier that nothing ever arrives on, so the bounded wait must expire, latch
@@ -245,17 +312,15 @@ int fp8q_weight_128x128(const uint16_t* w, int64_t N, int64_t K, uint8_t* q, flo
 size_t fp8q_gemm_workspace_size(int mode, int64_t M, int64_t N, int64_t K)
 {
     (void)mode;
-    (void)M;
-    (void)N;
-    (void)K;
-    return 0;
+    if (M <= 0 || N <= 0 || K < 256) return 0;   // one 128-K group: nothing to split
+    int sms = sm_count();
+    if (sms <= 0) sms = 148;
+    return sk_workspace_bytes(sms, 256);
 }
 
 int fp8_gemm_blockscaled(int mode, const uint8_t* A, const float* sA, const uint8_t* B, const float* sB, void* D,
                          int64_t M, int64_t N, int64_t K, void* workspace, size_t ws_bytes, fp8q_stream_t stream)
 {
-    (void)workspace;
-    (void)ws_bytes;
     if (mode != FP8Q_FPROP && mode != FP8Q_DGRAD && mode != FP8Q_WGRAD) return FP8Q_ERR_ARG;
     if (M < 0 || N < 0 || K < 0) return FP8Q_ERR_ARG;
     if (N % 128 != 0 || K % 128 != 0) return FP8Q_ERR_SHAPE;
@@ -270,9 +335,9 @@ int fp8_gemm_blockscaled(int mode, const uint8_t* A, const float* sA, const uint
     }
     const cudaStream_t st = (cudaStream_t)stream;
     switch (mode) {
-    case FP8Q_FPROP: return gemm_mode<kModeFprop>(A, sA, B, sB, D, M, N, K, st);
-    case FP8Q_DGRAD: return gemm_mode<kModeDgrad>(A, sA, B, sB, D, M, N, K, st);
-    default: return gemm_mode<kModeWgrad>(A, sA, B, sB, D, M, N, K, st);
+    case FP8Q_FPROP: return gemm_mode<kModeFprop>(A, sA, B, sB, D, M, N, K, st, workspace, ws_bytes);
+    case FP8Q_DGRAD: return gemm_mode<kModeDgrad>(A, sA, B, sB, D, M, N, K, st, workspace, ws_bytes);
+    default: return gemm_mode<kModeWgrad>(A, sA, B, sB, D, M, N, K, st, workspace, ws_bytes);
     }
 }
 

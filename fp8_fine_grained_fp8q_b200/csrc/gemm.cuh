@@ -38,7 +38,61 @@ struct GemmArgs {
     int32_t M;                // rows of A and D
     int32_t N;
     int32_t KB;               // K / 128
+    // Stream-K schedule (ws != nullptr): CTA c owns the (tile, 128-K group) units
+    // [units*c/G, units*(c+1)/G) of the tile-major unit space, G = gridDim.x.
+    float* ws;                // partial accumulators, one 128 x BN FP32 slot per CTA
+    unsigned long long* flags;   // per CTA: == stamp once its slot holds this launch's partial
+    unsigned long long stamp; // unique per launch, so flags never need resetting
+    int64_t units;            // tiles * KB
 };
+
+// One piece of work: groups [kb0, kb1) of tile `tile`.
+struct WorkItem {
+    int tile;
+    int kb0;
+    int kb1;
+};
+
+// Walks a CTA's work items.  Data-parallel: whole tiles c, c + G, ...  Stream-K: the CTA's
+// contiguous unit range cut at tile boundaries -- at most one leading item that starts
+// mid-tile (its partial goes to the workspace) and at most one trailing item that starts at
+// group 0 without reaching the end (it adds the later CTAs' partials, then stores the tile).
+struct WorkSched {
+    int64_t u, u_end;
+    int t;
+    bool sk;
+};
+
+__device__ __forceinline__ int64_t sk_begin(int64_t units, int c, int G) { return units * c / G; }
+
+__device__ __forceinline__ WorkSched sched_begin(const GemmArgs& a)
+{
+    WorkSched w;
+    w.sk = a.ws != nullptr;
+    w.t = (int)blockIdx.x;
+    w.u = w.sk ? sk_begin(a.units, (int)blockIdx.x, (int)gridDim.x) : 0;
+    w.u_end = w.sk ? sk_begin(a.units, (int)blockIdx.x + 1, (int)gridDim.x) : 0;
+    return w;
+}
+
+__device__ __forceinline__ bool sched_next(WorkSched& w, int num_tiles, int KB, WorkItem& it)
+{
+    if (!w.sk) {
+        if (w.t >= num_tiles) return false;
+        it.tile = w.t;
+        it.kb0 = 0;
+        it.kb1 = KB;
+        w.t += (int)gridDim.x;
+        return true;
+    }
+    if (w.u >= w.u_end) return false;
+    it.tile = (int)(w.u / KB);
+    it.kb0 = (int)(w.u - (int64_t)it.tile * KB);
+    const int64_t n = min((int64_t)(KB - it.kb0), w.u_end - w.u);
+    it.kb1 = it.kb0 + (int)n;
+    w.u += n;
+    return true;
+}
 
 template <int MODE, int BN, bool GROUPED>
 struct GemmShape {
@@ -55,7 +109,7 @@ struct GemmShape {
     static constexpr int kMaxGroups = 1024;
     static constexpr int kOffScales = kStages * kStageBytes;
     static constexpr int kOffBars = kOffScales + kScaleStages * BN * 4;
-    static constexpr int kNumBars = 2 * kStages + 4 + 2 * kScaleStages + 1;
+    static constexpr int kNumBars = 2 * kStages + 4 + 2 * kScaleStages + 2;
     static constexpr int kOffMisc = kOffBars + kNumBars * 8;
     static constexpr int kOffGroups = kOffMisc + 16;
     static constexpr int kSmemBytes = kOffGroups + (GROUPED ? 2 * (kMaxGroups + 1) * 4 : 0) + 1024;
@@ -127,6 +181,7 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
     const auto sfull_bar = [&](int s) { return bar0 + 8u * (2 * S::kStages + 4 + s); };
     const auto sempty_bar = [&](int s) { return bar0 + 8u * (2 * S::kStages + 4 + S::kScaleStages + s); };
     const uint32_t drain_bar = bar0 + 8u * (2 * S::kStages + 4 + 2 * S::kScaleStages);
+    const uint32_t parked_bar = drain_bar + 8u;   // stream-K: all promotion warps wrote the slot
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -146,6 +201,7 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
             mbar_init(sempty_bar(s), 8);
         }
         mbar_init(drain_bar, 1);
+        mbar_init(parked_bar, 8);
         misc[1] = 0;
         misc[2] = 0;
         fence_mbar_init();
@@ -211,10 +267,12 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
             int stage = 0, ss = 0;
             uint32_t phase = 0, sph = 0;
             bool ok = true;
-            for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
-                const TileInfo ti = decode_tile<GROUPED>(t, nb_tiles, BN, args, g_off, g_pre);
+            WorkSched ws = sched_begin(args);
+            WorkItem it;
+            while (ok && sched_next(ws, num_tiles, KB, it)) {
+                const TileInfo ti = decode_tile<GROUPED>(it.tile, nb_tiles, BN, args, g_off, g_pre);
                 const int brow = GROUPED ? ti.e * args.N + ti.n0 : ti.n0;
-                for (int kb = 0; kb < KB; ++kb) {
+                for (int kb = it.kb0; kb < it.kb1; ++kb) {
                     if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) { ok = false; break; }
                     const uint32_t sa = smem_u32(smem + stage * S::kStageBytes);
                     const uint32_t sb = sa + S::kABytes;
@@ -250,8 +308,10 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
             int stage = 0, tb = 0;
             uint32_t phase = 0, tph = 0;
             bool ok = true;
-            for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
-                for (int kb = 0; kb < KB; ++kb) {
+            WorkSched ws = sched_begin(args);
+            WorkItem it;
+            while (ok && sched_next(ws, num_tiles, KB, it)) {
+                for (int kb = it.kb0; kb < it.kb1; ++kb) {
                     if (!mbar_wait(tempty_bar(tb), tph ^ 1u, abort_flag)) { ok = false; break; }
                     if (!mbar_wait(full_bar(stage), phase, abort_flag)) { ok = false; break; }
                     tc_fence_after();
@@ -291,6 +351,7 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
         const int half = pw >> 2;             // columns [half*BN/2, (half+1)*BN/2)
         const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
         const int rit = quad * 32 + lane;     // row within the tile
+        const int ptid = pw * 32 + lane;      // promotion thread 0..255
         int tb = 0, ss = 0;
         uint32_t tph = 0, sph = 0;
         // Columns per TMEM load: 16 at BN = 256 (two chunks in flight still fit beside the 128
@@ -298,8 +359,11 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
         constexpr int kCW = 16;
         constexpr int kChunks = S::kHalf / kCW;
         float2 acc[S::kHalf / 2];
-        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
-            const TileInfo ti = decode_tile<GROUPED>(t, nb_tiles, BN, args, g_off, g_pre);
+        WorkSched wsched = sched_begin(args);
+        WorkItem it;
+        bool alive = true;
+        while (alive && sched_next(wsched, num_tiles, KB, it)) {
+            const TileInfo ti = decode_tile<GROUPED>(it.tile, nb_tiles, BN, args, g_off, g_pre);
             const int row = ti.row0 + rit;
             const bool in_a = row < args.M;
             const int ncol0 = ti.n0 + half * S::kHalf;
@@ -315,12 +379,12 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
             }
 #pragma unroll
             for (int i = 0; i < S::kHalf / 2; ++i) acc[i] = make_float2(0.0f, 0.0f);
-            float sa_next = in_a ? __ldg(sa_ptr) : 0.0f;
-            float sb_next = (MODE != kModeWgrad) ? __ldg(sb_ptr) : 1.0f;
+            float sa_next = in_a ? __ldg(sa_ptr + (size_t)it.kb0 * args.M) : 0.0f;
+            float sb_next = (MODE != kModeWgrad) ? __ldg(sb_ptr + (size_t)it.kb0 * sb_step) : 1.0f;
             bool ok = true;
-            for (int kb = 0; kb < KB; ++kb) {
+            for (int kb = it.kb0; kb < it.kb1; ++kb) {
                 const float sa = sa_next, sbv = sb_next;
-                if (kb + 1 < KB) {
+                if (kb + 1 < it.kb1) {
                     sa_next = in_a ? __ldg(sa_ptr + (size_t)(kb + 1) * args.M) : 0.0f;
                     if (MODE != kModeWgrad) sb_next = __ldg(sb_ptr + (size_t)(kb + 1) * sb_step);
                 }
@@ -388,6 +452,48 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                 if (++tb == 2) { tb = 0; tph ^= 1u; }
             }
             if (!ok) break;
+            if (wsched.sk && it.kb0 > 0) {
+                // Leading partial of a tile that another CTA finishes: park it in this CTA's slot.
+                // Only the same thread of the finishing CTA reads an entry back, so the slot is
+                // interleaved by promotion thread: each warp store moves 512 contiguous bytes.
+                float4* slot = reinterpret_cast<float4*>(args.ws + (size_t)blockIdx.x * (128 * BN)) + ptid;
+#pragma unroll
+                for (int j = 0; j < S::kHalf / 2; j += 2)
+                    __stcg(slot + (j / 2) * 256, make_float4(acc[j].x, acc[j].y, acc[j + 1].x, acc[j + 1].y));
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(parked_bar);
+                if (warp == 4 && lane == 0) {
+                    // A CTA parks at most one partial per launch (its first item): phase 0.
+                    if (mbar_wait(parked_bar, 0, abort_flag)) st_release_gpu(args.flags + blockIdx.x, args.stamp);
+                }
+                continue;
+            }
+            if (wsched.sk && it.kb1 < KB) {
+                // This CTA owns group 0 of the tile: add, in CTA order, the partials of the CTAs
+                // whose ranges start inside it (they computed them first, so the waits are short).
+                const int64_t tile_end = (int64_t)(it.tile + 1) * KB;
+                for (int j = (int)blockIdx.x + 1; j < (int)gridDim.x && sk_begin(args.units, j, gridDim.x) < tile_end;
+                     ++j) {
+                    bool ready = true;
+                    if (lane == 0) ready = spin_flag(args.flags + j, args.stamp, abort_flag);
+                    if (__shfl_sync(0xFFFFFFFFu, ready ? 1 : 0, 0) == 0) {
+                        alive = false;
+                        break;
+                    }
+                    __syncwarp();   // orders the lanes' loads of the slot after lane 0's acquire
+                    const float4* slot = reinterpret_cast<const float4*>(args.ws + (size_t)j * (128 * BN)) + ptid;
+#pragma unroll
+                    for (int q = 0; q < S::kHalf / 2; q += 2) {
+                        const float4 v = __ldcg(slot + (q / 2) * 256);
+                        acc[q].x += v.x;
+                        acc[q].y += v.y;
+                        acc[q + 1].x += v.z;
+                        acc[q + 1].y += v.w;
+                    }
+                }
+                if (!alive) break;
+            }
             // Epilogue: rows of this tile's group only.
             if (row < ti.row_end) {
                 if (MODE == kModeWgrad) {

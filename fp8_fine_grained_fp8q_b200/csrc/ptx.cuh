@@ -108,6 +108,38 @@ __device__ __forceinline__ void fence_proxy_async_smem()
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Publish / observe a 64-bit flag in global memory across CTAs (release / acquire, GPU scope).
+__device__ __forceinline__ void st_release_gpu(unsigned long long* p, unsigned long long v)
+{
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long ld_acquire_gpu(const unsigned long long* p)
+{
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Bounded spin until *p == want.  False (with the abort flag raised and FP8Q_DEV_TIMEOUT latched)
+// if the CTA is aborting or the limit expires.
+__device__ __forceinline__ bool spin_flag(const unsigned long long* p, unsigned long long want,
+                                          volatile int* abort_flag)
+{
+    if (ld_acquire_gpu(p) == want) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        __nanosleep(32);
+        if (ld_acquire_gpu(p) == want) return true;
+        if (*abort_flag) return false;
+        if ((it & 63u) == 0u && (globaltimer_ns() - t0 > kWaitLimitNs || it > kWaitLimitIters)) {
+            *abort_flag = 1;
+            latch_status(1 /* FP8Q_DEV_TIMEOUT */);
+            return false;
+        }
+    }
+}
+
 // Named barriers (ids 1..15; 0 is __syncthreads): `count` threads, a multiple of 32.
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count)
 {

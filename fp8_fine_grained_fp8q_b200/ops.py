@@ -145,10 +145,29 @@ def weight_128x128(w: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tens
 # GEMMs
 # ------------------------------------------------------------------------------------------ #
 
+_workspaces: dict = {}
+
+
+def gemm_workspace(mode: int, M: int, N: int, K: int, device: torch.device) -> torch.Tensor | None:
+    """The stream-K workspace a call of this size may use (cached per device; None if not needed)."""
+    nbytes = int(lib().fp8q_gemm_workspace_size(int(mode), M, N, K))
+    if nbytes == 0:
+        return None
+    key = device.index if device.index is not None else torch.cuda.current_device()
+    ws = _workspaces.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        _workspaces[key] = ws
+    return ws
+
+
 def gemm_blockscaled(mode: int, A: torch.Tensor, sA: torch.Tensor, B: torch.Tensor,
-                     sB: torch.Tensor, out: torch.Tensor | None = None):
+                     sB: torch.Tensor, out: torch.Tensor | None = None,
+                     workspace: torch.Tensor | None = None):
     """Block-scaled FP8 GEMM.  FPROP: B = W[N,K]; DGRAD: B = W[K,N]; WGRAD: B = X^T[N,K].
-    Returns D[M,N] (bf16, or fp32 for WGRAD)."""
+    Returns D[M,N] (bf16, or fp32 for WGRAD).  `workspace` (uint8, CUDA) enables the stream-K
+    schedule; by default a per-device workspace sized by fp8q_gemm_workspace_size is used.
+    A workspace must not be shared by GEMMs that may run concurrently."""
     _require(A, "A", torch.uint8, 2)
     _require(B, "B", torch.uint8, 2)
     _require(sA, "sA", torch.float32, 2)
@@ -160,9 +179,12 @@ def gemm_blockscaled(mode: int, A: torch.Tensor, sA: torch.Tensor, B: torch.Tens
         raise ValueError(f"inner dimensions differ: A has K={K}, B has {Kb}")
     dtype = torch.float32 if mode == WGRAD else torch.bfloat16
     out = _out(out, (M, N), dtype, A.device, "out")
+    if workspace is None:
+        workspace = gemm_workspace(mode, M, N, K, A.device)
+    ws_ptr, ws_bytes = (None, 0) if workspace is None else (_p(workspace), workspace.numel())
     _check("fp8_gemm_blockscaled",
            lib().fp8_gemm_blockscaled(int(mode), _p(A), _p(sA), _p(B), _p(sB), _p(out), M, N, K,
-                                      None, 0, _stream(A.device)))
+                                      ws_ptr, ws_bytes, _stream(A.device)))
     return out
 
 

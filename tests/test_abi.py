@@ -90,7 +90,9 @@ def test_gemm_host_checks(L):
     assert g(0, P(FAKE), P(FAKE), None, P(FAKE), P(FAKE), 128, 128, 128, None, 0, s) == ERR_ARG
     assert g(0, P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(MISALIGNED), 128, 128, 128, None, 0, s) == ERR_ALIGN
     assert g(0, *args, 1 << 31, 128, 128, None, 0, s) == ERR_UNSUPPORTED
-    assert L.fp8q_gemm_workspace_size(0, 4096, 2048, 7168) == 0
+    # Stream-K workspace: one 128 x 256 FP32 slot per CTA plus flags; none for a single K group.
+    assert L.fp8q_gemm_workspace_size(0, 4096, 2048, 7168) >= 148 * 128 * 256 * 4
+    assert L.fp8q_gemm_workspace_size(0, 4096, 2048, 128) == 0
 
 
 def test_grouped_host_checks(L):

@@ -21,9 +21,21 @@ pytestmark = pytest.mark.gpu
 FPROP, DGRAD, WGRAD = ops.FPROP, ops.DGRAD, ops.WGRAD
 
 
+# Kernel configurations: tile width x schedule (data-parallel whole tiles, or stream-K over
+# (tile, 128-K group) units with partials combined through the workspace).
+CONFIGS = {"n128-dp": ("128", "dp"), "n256-dp": ("256", "dp"),
+           "n128-sk": ("128", "sk"), "n256-sk": ("256", "sk")}
+
+
+def set_config(monkeypatch, cfg):
+    bn, sched = CONFIGS[cfg]
+    monkeypatch.setenv("FP8Q_GEMM_BN", bn)
+    monkeypatch.setenv("FP8Q_GEMM_SCHED", sched)
+
+
 def run_gemm(mode, A, sA, B, sB, bn=None, monkeypatch=None):
     if bn is not None:
-        monkeypatch.setenv("FP8Q_GEMM_BN", str(bn))
+        set_config(monkeypatch, bn)
     M = A.shape[0]
     N = B.shape[1] if mode == DGRAD else B.shape[0]
     dtype = torch.float32 if mode == WGRAD else torch.bfloat16
@@ -63,7 +75,7 @@ def exact_fprop(M, N, K, seed):
     return X, W, exact
 
 
-@pytest.mark.parametrize("bn", [128, 256])
+@pytest.mark.parametrize("bn", list(CONFIGS))
 @pytest.mark.parametrize("M,N,K", [(128, 256, 256), (200, 512, 384), (1, 256, 128), (384, 256, 1024)])
 def test_exact_fprop(M, N, K, bn, monkeypatch):
     X, W, exact = exact_fprop(M, N, K, seed=M + N + K)
@@ -78,7 +90,7 @@ def test_exact_fprop(M, N, K, bn, monkeypatch):
     assert np.array_equal(got, exact)
 
 
-@pytest.mark.parametrize("bn", [128, 256])
+@pytest.mark.parametrize("bn", list(CONFIGS))
 @pytest.mark.parametrize("M,N,K", [(128, 256, 256), (260, 512, 384)])
 def test_exact_dgrad(M, N, K, bn, monkeypatch):
     # dX[M,N] = dY[M,K] W[K,N]; W is the forward weight [out=K, in=N].
@@ -101,7 +113,7 @@ def test_exact_dgrad(M, N, K, bn, monkeypatch):
     assert np.array_equal(got, exact)
 
 
-@pytest.mark.parametrize("bn", [128, 256])
+@pytest.mark.parametrize("bn", list(CONFIGS))
 @pytest.mark.parametrize("T,Cout,Cin", [(128, 128, 256), (512, 384, 512)])
 def test_exact_wgrad(T, Cout, Cin, bn, monkeypatch):
     # dW[Cout,Cin] = dY[T,Cout]^T X[T,Cin]; FP32 output, so larger sums stay exact.
@@ -136,7 +148,7 @@ def test_tiny_fprop_workload():
     check_gemm(got, ref, S, "tiny fprop 256x512x512")
 
 
-@pytest.mark.parametrize("bn", [128, 256])
+@pytest.mark.parametrize("bn", list(CONFIGS))
 @pytest.mark.parametrize("M,N,K", [(200, 256, 384), (517, 512, 1024), (1, 256, 256)])
 def test_fprop_ragged(M, N, K, bn, monkeypatch):
     X = synth.activations_channel_outliers(M, K, seed=M + K)
@@ -147,7 +159,7 @@ def test_fprop_ragged(M, N, K, bn, monkeypatch):
     check_gemm(run_gemm(FPROP, xq, xs, wq, ws, bn, monkeypatch), ref, S, f"fprop {M}x{N}x{K}")
 
 
-@pytest.mark.parametrize("bn", [128, 256])
+@pytest.mark.parametrize("bn", list(CONFIGS))
 @pytest.mark.parametrize("M,N,K", [(256, 512, 256), (333, 768, 640)])
 def test_dgrad_ragged(M, N, K, bn, monkeypatch):
     dY = synth.output_grad(M, K, seed=M + K)
@@ -158,7 +170,7 @@ def test_dgrad_ragged(M, N, K, bn, monkeypatch):
     check_gemm(run_gemm(DGRAD, gq, gs, wq, ws, bn, monkeypatch), ref, S, f"dgrad {M}x{N}x{K}")
 
 
-@pytest.mark.parametrize("bn", [128, 256])
+@pytest.mark.parametrize("bn", list(CONFIGS))
 @pytest.mark.parametrize("T,Cout,Cin", [(512, 256, 512), (384, 384, 768)])
 def test_wgrad(T, Cout, Cin, bn, monkeypatch):
     dY = synth.output_grad(T, Cout, seed=T + Cout)
@@ -245,19 +257,20 @@ def test_full_fprop_mla(N):
     sampled_check(FPROP, xq, xs, wq, ws, got, f"fprop MLA 4096x{N}x7168")
 
 
+@pytest.mark.parametrize("cfg", list(CONFIGS))
 @pytest.mark.parametrize("mode", [FPROP, DGRAD, WGRAD])
-def test_full_size_deterministic_and_tile_width_invariant(mode, monkeypatch):
-    """Repeated launches are bitwise identical, and both tile widths give the same bits (each
-    output element is folded in the same K-group order either way).  Catches pipeline races,
-    e.g. a shared-memory buffer refilled by the async proxy while threads still read it."""
+def test_full_size_every_config_deterministic_and_within_tolerance(mode, cfg, monkeypatch):
+    """Each kernel configuration is run twice at full size: the launches must be bitwise
+    identical (a race would show here -- e.g. a shared-memory buffer refilled by the async proxy
+    while threads still read it, or a stream-K partial read before it is published), and the
+    result must match the oracle on the sampled entries."""
     q = quantised_layer()
     (a, sa), (b, sb) = {FPROP: (q["X"], q["W"]), DGRAD: (q["dY"], q["W"]),
                         WGRAD: (q["dYt"], q["Xt"])}[mode]
     A, SA, B, SB = u8_dev(a), f32_dev(sa), u8_dev(b), f32_dev(sb)
-    outs = []
-    for bn in (128, 256, 128, 256):
-        monkeypatch.setenv("FP8Q_GEMM_BN", str(bn))
-        outs.append(ops.gemm_blockscaled(mode, A, SA, B, SB).clone())
+    set_config(monkeypatch, cfg)
+    first = ops.gemm_blockscaled(mode, A, SA, B, SB).clone()
+    second = ops.gemm_blockscaled(mode, A, SA, B, SB)
     assert ops.device_status() == ops.DEV_OK
-    for o in outs[1:]:
-        assert torch.equal(o, outs[0])
+    assert torch.equal(first, second)
+    sampled_check(mode, a, sa, b, sb, host(first), f"mode {mode} {cfg}")
