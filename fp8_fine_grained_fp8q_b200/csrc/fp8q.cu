@@ -240,6 +240,38 @@ __global__ void selftest_wait_kernel(uint64_t limit_ns)
     if (threadIdx.x == 0) mbar_wait_slow(smem_u32(&bar), 0, &abort_flag, limit_ns);
 }
 
+// ------------------------------------------------------------------------------------------
+// Allocation-free GEMM: the stream-K scratch lives in a file-scope device array instead of a
+// caller workspace.  It holds the slots and flags of kNoallocMaxCtas persistent CTAs of
+// 256-wide tiles (about 20 MiB), is present on every GPU that loads this library, and lives
+// until the process exits.
+// ------------------------------------------------------------------------------------------
+constexpr int kNoallocMaxCtas = 160;
+constexpr size_t kNoallocScratchBytes =
+    (size_t)kNoallocMaxCtas * 128 * 256 * sizeof(float) + (((size_t)kNoallocMaxCtas * sizeof(uint64_t) + 255) & ~(size_t)255);
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+
+// Device address of g_noalloc_scratch on the current device.  In host code the array's name is
+// only a host-side stand-in, so the address is looked up once per device (with that device
+// current) and cached.  Returns nullptr if the lookup fails.
+void* noalloc_scratch()
+{
+    static void* addr[kMaxDevices] = {nullptr};
+    static std::mutex lock;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> guard(lock);
+    if (addr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        addr[dev] = p;
+    }
+    return addr[dev];
+}
+
 }  // namespace
 
 // ==========================================================================================
@@ -257,6 +289,7 @@ const char* fp8q_status_string(int status)
     case FP8Q_ERR_CUDA: return "CUDA error";
     case FP8Q_ERR_UNSUPPORTED: return "size or configuration not supported by this build";
     case FP8Q_ERR_DEVICE: return "error reported by the device";
+    case FP8Q_ERR_SCRATCH: return "the allocation-free GEMM needs more scratch than its fixed array holds";
     default: return "unknown status";
     }
 }
@@ -339,6 +372,21 @@ int fp8_gemm_blockscaled(int mode, const uint8_t* A, const float* sA, const uint
     case FP8Q_DGRAD: return gemm_mode<kModeDgrad>(A, sA, B, sB, D, M, N, K, st, workspace, ws_bytes);
     default: return gemm_mode<kModeWgrad>(A, sA, B, sB, D, M, N, K, st, workspace, ws_bytes);
     }
+}
+
+int fp8_gemm_blockscaled_noalloc(int mode, const uint8_t* A, const float* sA, const uint8_t* B, const float* sB,
+                                 void* D, int64_t M, int64_t N, int64_t K, fp8q_stream_t stream)
+{
+    // The stream-K schedule needs one slot per persistent CTA (one per SM); the data-parallel
+    // schedule needs none.  Refuse problems whose scratch would not fit the fixed array.
+    const size_t need = fp8q_gemm_workspace_size(mode, M, N, K);
+    if (need > kNoallocScratchBytes) return FP8Q_ERR_SCRATCH;
+    void* scratch = nullptr;
+    if (need > 0) {
+        scratch = noalloc_scratch();
+        if (!scratch) return FP8Q_ERR_CUDA;
+    }
+    return fp8_gemm_blockscaled(mode, A, sA, B, sB, D, M, N, K, scratch, scratch ? kNoallocScratchBytes : 0, stream);
 }
 
 int fp8_grouped_gemm_blockscaled(const uint8_t* A, const float* sA, const uint8_t* B, const float* sB,

@@ -63,7 +63,8 @@ enum {
     FP8Q_ERR_ALIGN = 3,        /* a data pointer is not 16-byte aligned */
     FP8Q_ERR_CUDA = 4,         /* a CUDA runtime or driver call failed (no device, launch error) */
     FP8Q_ERR_UNSUPPORTED = 5,  /* a size beyond what this build supports (see each call) */
-    FP8Q_ERR_DEVICE = 6        /* reported by fp8q_device_status: an error latched on the device */
+    FP8Q_ERR_DEVICE = 6,       /* reported by fp8q_device_status: an error latched on the device */
+    FP8Q_ERR_SCRATCH = 7       /* fp8_gemm_blockscaled_noalloc: scratch need exceeds its fixed array */
 };
 
 /* Device status word values (what fp8q_device_status writes to *out). */
@@ -136,6 +137,30 @@ FP8Q_API int fp8_gemm_blockscaled(int mode, const uint8_t* A, const float* sA, c
                          void* workspace, size_t ws_bytes, fp8q_stream_t stream);
 
 FP8Q_API size_t fp8q_gemm_workspace_size(int mode, int64_t M, int64_t N, int64_t K);
+
+/*
+ * fp8_gemm_blockscaled without a workspace argument, for callers that may not allocate device
+ * memory themselves: a plugin running inside a host framework that owns the device memory pool
+ * and gives its kernels only their inputs and outputs, or a latency-critical path that cannot
+ * afford cudaMalloc's implicit device-wide synchronisation.  (This entry point has no
+ * counterpart on the pages; it is packaging, not part of the method.)
+ *
+ * Same arguments, results and requirements as fp8_gemm_blockscaled.  The stream-K scratch that
+ * call would take from `workspace` comes instead from a fixed device array inside the library:
+ * room for the partial slots and flags of 160 persistent CTAs of 256-wide tiles, about 20 MiB,
+ * held by every GPU that loads the library until the process exits.  Problems whose scratch
+ * would exceed it (a device with more than 160 SMs) get FP8Q_ERR_SCRATCH.  No call allocates or
+ * frees anything.
+ * - The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
+ *   that device current) and caches it; make that first call before any stream capture.
+ * - Every call shares the one array per device and leaves its contents behind.  Nothing in it
+ *   needs clearing: each launch stamps its flags with a value no earlier launch used.
+ * - Calls whose GPU work overlaps (on different streams, or from different threads) race on the
+ *   shared scratch and give wrong results; order them on one stream or with events.
+ */
+FP8Q_API int fp8_gemm_blockscaled_noalloc(int mode, const uint8_t* A, const float* sA, const uint8_t* B,
+                                          const float* sB, void* D, int64_t M, int64_t N, int64_t K,
+                                          fp8q_stream_t stream);
 
 /*
  * Grouped (MoE expert) block-scaled FP8 Fprop over ragged row groups: the rows of A are sorted
