@@ -3,10 +3,10 @@
 
 Workload (one "step"): the DeepSeek-V3 expert-FFN up-projection linear layer with 4096 tokens,
 C_in = 7168, C_out = 2048, bf16 operands resident in HBM:
-    act 1x128 (X)  -> weight 128x128 (W) -> Fprop  Y  = X W^T      (bf16 [4096, 2048])
-    act 1x128 (dY)                      -> Dgrad  dX = dY W        (bf16 [4096, 7168])
-    act 128x1^T (X), act 128x1^T (dY)   -> Wgrad  dW = dY^T X      (fp32 [2048, 7168])
-8 kernel launches.  value = GEMM FLOPs (3 x 2*4096*2048*7168) / device time of the step.
+    act 1x128 + 128x1^T (X, one pass) -> weight 128x128 (W) -> Fprop Y = X W^T (bf16 [4096, 2048])
+    act 1x128 + 128x1^T (dY, one pass)                     -> Dgrad dX = dY W  (bf16 [4096, 7168])
+                                                              Wgrad dW = dY^T X (fp32 [2048, 7168])
+6 kernel launches (8 with --separate-quant, which quantises each form in its own launch).  value = GEMM FLOPs (3 x 2*4096*2048*7168) / device time of the step.
 L2 is flushed (256 MiB write) between steps, outside the timed step.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
@@ -35,14 +35,15 @@ T_TOK, C_IN, C_OUT = 4096, 7168, 2048
 GEMM_FLOP = 2.0 * T_TOK * C_OUT * C_IN           # each of Fprop, Dgrad, Wgrad
 STEP_FLOP = 3.0 * GEMM_FLOP
 METRIC = ("block-scaled FP8 GEMM TFLOP/s (% dense FP8 peak); quantizer GB/s (% HBM)")
-WORKLOAD = ("FP8 linear layer training GEMMs (act 1x128 + weight 128x128 + Fprop, act 1x128 + "
-            "Dgrad, 2x act 128x1-transposed + Wgrad), tokens 4096, C_in 7168, C_out 2048")
+WORKLOAD = ("FP8 linear layer training GEMMs (act 1x128 + 128x1-transposed of X and of dY, "
+            "weight 128x128, Fprop, Dgrad, Wgrad), tokens 4096, C_in 7168, C_out 2048")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP8_OVER_BF16 = 2.0                              # nominal dense ratio (4.5 / 2.25 PFLOP/s)
 
 # Algorithmic bytes per element: bf16 read (2) + code write (1) + one fp32 scale per group.
 QB_1x128 = 2 + 1 + 4 / 128
 QB_128x128 = 2 + 1 + 4 / (128 * 128)
+QB_DUAL = 2 + 2 * (1 + 4 / 128)                  # one read, both code sets and scale sets
 
 
 def load_peaks():
@@ -139,8 +140,10 @@ class ClockSampler:
 # ------------------------------------------------------------------------------------------ #
 # GPU arm
 # ------------------------------------------------------------------------------------------ #
-OPS = ["act_1x128_X", "weight_128x128_W", "gemm_fprop", "act_1x128_dY", "gemm_dgrad",
-       "act_128x1t_X", "act_128x1t_dY", "gemm_wgrad"]
+OPS_FUSED = ["act_dual_X", "weight_128x128_W", "gemm_fprop", "act_dual_dY", "gemm_dgrad",
+             "gemm_wgrad"]
+OPS_SEPARATE = ["act_1x128_X", "weight_128x128_W", "gemm_fprop", "act_1x128_dY", "gemm_dgrad",
+                "act_128x1t_X", "act_128x1t_dY", "gemm_wgrad"]
 
 
 def make_buffers(torch, dev):
@@ -164,23 +167,34 @@ def make_buffers(torch, dev):
     return host, t, b
 
 
-def step_ops(ops, t, b):
-    """The step as a list of zero-argument launches (all on torch's current stream)."""
-    return [
-        lambda: ops.act_1x128(t["X"], b["Xq"], b["sX"]),
-        lambda: ops.weight_128x128(t["W"], b["Wq"], b["sW"]),
-        lambda: ops.gemm_blockscaled(ops.FPROP, b["Xq"], b["sX"], b["Wq"], b["sW"], b["Y"]),
-        lambda: ops.act_1x128(t["dY"], b["dYq"], b["sdY"]),
-        lambda: ops.gemm_blockscaled(ops.DGRAD, b["dYq"], b["sdY"], b["Wq"], b["sW"], b["dX"]),
-        lambda: ops.act_128x1_transposed(t["X"], b["Xtq"], b["sXt"]),
-        lambda: ops.act_128x1_transposed(t["dY"], b["dYtq"], b["sdYt"]),
-        lambda: ops.gemm_blockscaled(ops.WGRAD, b["dYtq"], b["sdYt"], b["Xtq"], b["sXt"], b["dW"]),
-    ]
+def step_ops(ops, t, b, separate=False):
+    """The step as (names, zero-argument launches), all on torch's current stream.  By default
+    X and dY are quantised to both forms in one pass each (act_dual); separate=True runs the
+    1x128 and 128x1-transposed quantisers as their own launches."""
+    gemms = {
+        "gemm_fprop": lambda: ops.gemm_blockscaled(ops.FPROP, b["Xq"], b["sX"], b["Wq"], b["sW"], b["Y"]),
+        "gemm_dgrad": lambda: ops.gemm_blockscaled(ops.DGRAD, b["dYq"], b["sdY"], b["Wq"], b["sW"], b["dX"]),
+        "gemm_wgrad": lambda: ops.gemm_blockscaled(ops.WGRAD, b["dYtq"], b["sdYt"], b["Xtq"], b["sXt"], b["dW"]),
+    }
+    quant = {
+        "act_dual_X": lambda: ops.act_dual(t["X"], b["Xq"], b["sX"], b["Xtq"], b["sXt"]),
+        "act_dual_dY": lambda: ops.act_dual(t["dY"], b["dYq"], b["sdY"], b["dYtq"], b["sdYt"]),
+        "act_1x128_X": lambda: ops.act_1x128(t["X"], b["Xq"], b["sX"]),
+        "act_1x128_dY": lambda: ops.act_1x128(t["dY"], b["dYq"], b["sdY"]),
+        "act_128x1t_X": lambda: ops.act_128x1_transposed(t["X"], b["Xtq"], b["sXt"]),
+        "act_128x1t_dY": lambda: ops.act_128x1_transposed(t["dY"], b["dYtq"], b["sdYt"]),
+        "weight_128x128_W": lambda: ops.weight_128x128(t["W"], b["Wq"], b["sW"]),
+    }
+    names = OPS_SEPARATE if separate else OPS_FUSED
+    table = {**gemms, **quant}
+    return names, [table[n] for n in names]
 
 
 def op_work():
     """Algorithmic work per launch: ('flop', F) or ('bytes', B)."""
     return {
+        "act_dual_X": ("bytes", T_TOK * C_IN * QB_DUAL),
+        "act_dual_dY": ("bytes", T_TOK * C_OUT * QB_DUAL),
         "act_1x128_X": ("bytes", T_TOK * C_IN * QB_1x128),
         "weight_128x128_W": ("bytes", C_OUT * C_IN * QB_128x128),
         "gemm_fprop": ("flop", GEMM_FLOP),
@@ -201,7 +215,7 @@ def run_ours(args, rank, world, dist):
     dev = torch.device("cuda", local)
     ops.lib()                                      # fail loudly if the library is missing
     host, t, b = make_buffers(torch, dev)
-    launches = step_ops(ops, t, b)
+    OPS, launches = step_ops(ops, t, b, separate=args.separate_quant)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     torch.cuda.synchronize()
 
@@ -416,6 +430,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle CPU work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--separate-quant", action="store_true",
+                    help="quantise X and dY with separate 1x128 and 128x1 launches")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be at least 3")

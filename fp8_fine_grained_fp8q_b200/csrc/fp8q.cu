@@ -307,10 +307,11 @@ int fp8q_act_1x128(const uint16_t* x, int64_t M, int64_t K, uint8_t* q, float* s
     if (sms <= 0) return FP8Q_ERR_CUDA;
     constexpr int kUnr = 4;
     const int64_t ntiles = M * (K / 128);
-    const int64_t want = (ntiles + 16 * kUnr - 1) / (16 * kUnr);   // blocks of 16 half-warps
+    if (ntiles >= (1ll << 31) || M >= (1ll << 31)) return FP8Q_ERR_UNSUPPORTED;
+    const int64_t want = (ntiles + 32 * kUnr - 1) / (32 * kUnr);   // blocks of 32 eight-lane groups
     const int64_t cap = (int64_t)sms * 8;
     const int grid = (int)(want < cap ? want : cap);
-    act_1x128_kernel<kUnr><<<grid, 256, 0, (cudaStream_t)stream>>>(x, q, s, M, K);
+    act_1x128_kernel<kUnr><<<grid, 256, 0, (cudaStream_t)stream>>>(x, q, s, (int)M, (int)K);
     return launch_status();
 }
 
@@ -325,6 +326,21 @@ int fp8q_act_128x1_transposed(const uint16_t* x, int64_t T, int64_t C, uint8_t* 
     if (T / 128 > 65535 || C / 64 > 0x7FFFFFFF) return FP8Q_ERR_UNSUPPORTED;
     const dim3 grid((unsigned)(C / 64), (unsigned)(T / 128));
     act_128x1_t_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(x, qt, s, T, C);
+    return launch_status();
+}
+
+int fp8q_act_dual(const uint16_t* x, int64_t T, int64_t C, uint8_t* q, float* s, uint8_t* qt, float* st,
+                  fp8q_stream_t stream)
+{
+    if (T < 0 || C < 0) return FP8Q_ERR_ARG;
+    if (T % 128 != 0 || C % 128 != 0) return FP8Q_ERR_SHAPE;
+    if (T == 0 || C == 0) return FP8Q_OK;
+    if (!x || !q || !s || !qt || !st) return FP8Q_ERR_ARG;
+    if (!aligned16(x) || !aligned16(q) || !aligned16(s) || !aligned16(qt) || !aligned16(st))
+        return FP8Q_ERR_ALIGN;
+    if (T / 128 > 65535 || C / 128 > 0x7FFFFFFF) return FP8Q_ERR_UNSUPPORTED;
+    const dim3 grid((unsigned)(C / 128), (unsigned)(T / 128));
+    act_dual_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(x, q, s, qt, st, T, C);
     return launch_status();
 }
 

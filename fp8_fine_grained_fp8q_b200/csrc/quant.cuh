@@ -60,45 +60,58 @@ __device__ __forceinline__ void group_scale(float amax, float& s, float& inv)
 }
 
 // ------------------------------------------------------------------------------------------
-// 1x128: x[M,K] -> q[M,K], s[K/128][M].  A half-warp owns one tile (16 lanes x 16 B = 256 B of
-// bf16); each lane keeps UNR tiles' loads in flight.  Tiles are visited in row-major order so
-// the reads stream through HBM sequentially.
+// 1x128: x[M,K] -> q[M,K], s[K/128][M].  Eight lanes own one tile (8 x 32 B = 256 B of bf16,
+// 16 values per lane), so a warp covers 4 consecutive tiles = 1 KB of contiguous input per
+// load; the max-abs needs 3 shuffle levels.  Each lane keeps UNR tile-groups of loads in
+// flight.  Tiles are visited row-major so the reads stream through HBM sequentially; all index
+// arithmetic is 32-bit (the host guarantees M * K/128 < 2^31).
 // ------------------------------------------------------------------------------------------
+__device__ __forceinline__ float amax16(const uint4& a, const uint4& b)
+{
+    return fmaxf(amax8(a), amax8(b));
+}
+
 template <int UNR>
 __global__ void __launch_bounds__(256) act_1x128_kernel(const uint16_t* __restrict__ x,
                                                         uint8_t* __restrict__ q,
-                                                        float* __restrict__ s, int64_t M, int64_t K)
+                                                        float* __restrict__ s, int M, int K)
 {
-    const int64_t KB = K >> 7;
-    const int64_t ntiles = M * KB;
-    const int sub = threadIdx.x & 15;
-    const int64_t hw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 4;
-    const int64_t nhw = ((int64_t)gridDim.x * blockDim.x) >> 4;
+    const uint32_t KB = (uint32_t)K >> 7;
+    const uint32_t ntiles = (uint32_t)M * KB;
+    const uint32_t sub = threadIdx.x & 7;                       // lane within the tile
+    const uint32_t g8 = ((uint32_t)blockIdx.x * blockDim.x + threadIdx.x) >> 3;   // 8-lane group
+    const uint32_t ng8 = ((uint32_t)gridDim.x * blockDim.x) >> 3;
 
-    for (int64_t base = hw; base < ntiles; base += nhw * UNR) {
-        uint4 v[UNR];
+    for (uint32_t base = g8; base < ntiles; base += ng8 * UNR) {
+        uint4 v[UNR][2];
 #pragma unroll
         for (int u = 0; u < UNR; ++u) {
-            const int64_t t = base + (int64_t)u * nhw;
-            v[u] = make_uint4(0u, 0u, 0u, 0u);
+            const uint32_t t = base + (uint32_t)u * ng8;
+            v[u][0] = make_uint4(0u, 0u, 0u, 0u);
+            v[u][1] = make_uint4(0u, 0u, 0u, 0u);
             if (t < ntiles) {
-                const int64_t m = t / KB, kb = t - m * KB;
-                v[u] = __ldg(reinterpret_cast<const uint4*>(x + m * K + kb * 128) + sub);
+                // Tile t = (m, kb) row-major is the 256 B at element offset t * 128.
+                const uint4* p = reinterpret_cast<const uint4*>(x + (size_t)t * 128) + 2 * sub;
+                v[u][0] = __ldg(p);
+                v[u][1] = __ldg(p + 1);
             }
         }
 #pragma unroll
         for (int u = 0; u < UNR; ++u) {
-            const int64_t t = base + (int64_t)u * nhw;
-            float amax = amax8(v[u]);
-            // All 32 lanes take part in the shuffles even when one half-warp has no tile.
+            const uint32_t t = base + (uint32_t)u * ng8;
+            float amax = amax16(v[u][0], v[u][1]);
+            // All 32 lanes take part in the shuffles even when an 8-lane group has no tile.
 #pragma unroll
-            for (int o = 8; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+            for (int o = 4; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
             float sc, inv;
             group_scale(amax, sc, inv);
             if (t < ntiles) {
-                const int64_t m = t / KB, kb = t - m * KB;
-                reinterpret_cast<uint2*>(q + m * K + kb * 128)[sub] = quant8(v[u], inv);
-                if (sub == 0) s[kb * M + m] = sc;
+                const uint2 lo = quant8(v[u][0], inv), hi = quant8(v[u][1], inv);
+                reinterpret_cast<uint4*>(q + (size_t)t * 128)[sub] = make_uint4(lo.x, lo.y, hi.x, hi.y);
+                if (sub == 0) {
+                    const uint32_t m = t / KB, kb = t - m * KB;
+                    s[(size_t)kb * M + m] = sc;
+                }
             }
         }
     }
@@ -106,83 +119,177 @@ __global__ void __launch_bounds__(256) act_1x128_kernel(const uint16_t* __restri
 
 // ------------------------------------------------------------------------------------------
 // 128x1 with transposed output: x[T,C] -> qt[C,T], s[T/128][C].  One CTA per 128-token x
-// 64-channel tile: coalesced 16 B row loads into shared memory, column max-abs by warps that
-// each scan every 8th token (lanes = channel pairs, conflict-free), then each thread writes
-// 16 consecutive tokens of one channel as one 16 B store.
+// 64-channel tile.  Warp w reads tokens 16w .. 16w+15; lane l owns channels 2l, 2l+1, so each
+// 4-byte load of the warp is one coalesced 128-byte row segment and the thread ends up holding
+// its 16 tokens x 2 channels in registers (the transpose happens in registers, not in shared
+// memory).  Only the per-channel max-abs crosses warps, through a small shared reduction; then
+// each thread converts its values and writes 16 consecutive tokens of each of its two channels
+// as one 16-byte store each.
 // ------------------------------------------------------------------------------------------
 constexpr int kT1Tok = 128;
 constexpr int kT1Ch = 64;
-constexpr int kT1Pitch = kT1Ch + 8;   // bf16 elements per shared row (144 B, 16 B aligned)
 
 __global__ void __launch_bounds__(256) act_128x1_t_kernel(const uint16_t* __restrict__ x,
                                                           uint8_t* __restrict__ qt,
                                                           float* __restrict__ s, int64_t T, int64_t C)
 {
-    __shared__ __align__(16) uint16_t tile[kT1Tok][kT1Pitch];
     __shared__ float red[8][kT1Ch];
     __shared__ float inv_c[kT1Ch];
 
     const int64_t c0 = (int64_t)blockIdx.x * kT1Ch;
     const int64_t tb = blockIdx.y;
     const int64_t t0 = tb * kT1Tok;
-    const int tid = threadIdx.x;
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    uint4 v[4];
+    // Tokens t0 + 16w + i, channels c0 + 2*lane (low half) and c0 + 2*lane + 1 (high half).
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(x + (t0 + 16 * w) * C + c0) + lane;
+    uint32_t v[16];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int idx = tid + 256 * i;
-        const int r = idx >> 3, c8 = idx & 7;
-        v[i] = __ldg(reinterpret_cast<const uint4*>(x + (t0 + r) * C + c0) + c8);
-    }
+    for (int i = 0; i < 16; ++i) v[i] = __ldg(src + (size_t)i * (size_t)(C >> 1));
+    float m0 = 0.0f, m1 = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int idx = tid + 256 * i;
-        const int r = idx >> 3, c8 = idx & 7;
-        *reinterpret_cast<uint4*>(&tile[r][c8 * 8]) = v[i];
+    for (int i = 0; i < 16; ++i) {
+        m0 = fmaxf(m0, fabsf(bf16_lo(v[i])));
+        m1 = fmaxf(m1, fabsf(bf16_hi(v[i])));
     }
+    red[w][2 * lane] = m0;
+    red[w][2 * lane + 1] = m1;
     __syncthreads();
-
-    {
-        const int w = tid >> 5, lane = tid & 31;
-        float m0 = 0.0f, m1 = 0.0f;
+    if (threadIdx.x < kT1Ch) {
+        float a = red[0][threadIdx.x];
 #pragma unroll
-        for (int i = 0; i < kT1Tok / 8; ++i) {
-            const uint32_t pr = *reinterpret_cast<const uint32_t*>(&tile[8 * i + w][2 * lane]);
-            m0 = fmaxf(m0, fabsf(bf16_lo(pr)));
-            m1 = fmaxf(m1, fabsf(bf16_hi(pr)));
-        }
-        red[w][2 * lane] = m0;
-        red[w][2 * lane + 1] = m1;
-    }
-    __syncthreads();
-    if (tid < kT1Ch) {
-        float a = red[0][tid];
-#pragma unroll
-        for (int w = 1; w < 8; ++w) a = fmaxf(a, red[w][tid]);
+        for (int k = 1; k < 8; ++k) a = fmaxf(a, red[k][threadIdx.x]);
         float sc, inv;
         group_scale(a, sc, inv);
-        s[tb * C + c0 + tid] = sc;
-        inv_c[tid] = inv;
+        s[tb * C + c0 + threadIdx.x] = sc;
+        inv_c[threadIdx.x] = inv;
     }
     __syncthreads();
-
+    const float inv0 = inv_c[2 * lane], inv1 = inv_c[2 * lane + 1];
+    uint32_t q0[4], q1[4];
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-        const int item = tid + 256 * j;
-        const int c = item & (kT1Ch - 1), seg = item >> 6;   // seg: 16-token segment 0..7
-        const float inv = inv_c[c];
-        uint32_t w4[4];
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            const int tk = seg * 16 + 4 * p;
-            const float f0 = __fmul_rn(__uint_as_float((uint32_t)tile[tk + 0][c] << 16), inv);
-            const float f1 = __fmul_rn(__uint_as_float((uint32_t)tile[tk + 1][c] << 16), inv);
-            const float f2 = __fmul_rn(__uint_as_float((uint32_t)tile[tk + 2][c] << 16), inv);
-            const float f3 = __fmul_rn(__uint_as_float((uint32_t)tile[tk + 3][c] << 16), inv);
-            w4[p] = e4m3x2(f0, f1) | (e4m3x2(f2, f3) << 16);
-        }
-        *reinterpret_cast<uint4*>(qt + (c0 + c) * T + t0 + seg * 16) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    for (int p = 0; p < 4; ++p) {
+        q0[p] = e4m3x2(__fmul_rn(bf16_lo(v[4 * p + 0]), inv0), __fmul_rn(bf16_lo(v[4 * p + 1]), inv0)) |
+                (e4m3x2(__fmul_rn(bf16_lo(v[4 * p + 2]), inv0), __fmul_rn(bf16_lo(v[4 * p + 3]), inv0)) << 16);
+        q1[p] = e4m3x2(__fmul_rn(bf16_hi(v[4 * p + 0]), inv1), __fmul_rn(bf16_hi(v[4 * p + 1]), inv1)) |
+                (e4m3x2(__fmul_rn(bf16_hi(v[4 * p + 2]), inv1), __fmul_rn(bf16_hi(v[4 * p + 3]), inv1)) << 16);
     }
+    uint8_t* dst = qt + (c0 + 2 * lane) * T + t0 + 16 * w;
+    *reinterpret_cast<uint4*>(dst) = make_uint4(q0[0], q0[1], q0[2], q0[3]);
+    *reinterpret_cast<uint4*>(dst + T) = make_uint4(q1[0], q1[1], q1[2], q1[3]);
+}
+
+// ------------------------------------------------------------------------------------------
+// Both activation forms in one pass: x[T,C] -> (q[T,C], s[C/128][T]) as the 1x128 kernel and
+// (qt[C,T], st[T/128][C]) as the 128x1 kernel, reading x once.  One CTA per 128-token x
+// 128-channel tile, which is a whole group in both directions.  Warp w holds tokens
+// 16w .. 16w+15; lane l holds channels 4l .. 4l+3 (one 8-byte load per token row, 256 B per
+// warp instruction).  Column max-abs: per thread over its 16 tokens, then across warps in
+// shared memory.  Row max-abs: a shuffle reduce-scatter (16 -> 8 -> 4 -> 2 -> 1 values per
+// lane, then one all-reduce step) leaves the maximum of row 16w + (l >> 1) on lanes 2r, 2r+1.
+// Codes: rows as 4-byte stores (128 B per warp row), columns as 16-byte stores of 16 tokens.
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256, 3) act_dual_kernel(const uint16_t* __restrict__ x,
+                                                       uint8_t* __restrict__ q, float* __restrict__ s,
+                                                       uint8_t* __restrict__ qt, float* __restrict__ st,
+                                                       int64_t T, int64_t C)
+{
+    __shared__ __align__(16) float red[8][128];
+    __shared__ __align__(16) float inv_c[128];
+
+    const int64_t cb = blockIdx.x, tb = blockIdx.y;
+    const int64_t c0 = cb * 128, t0 = tb * 128;
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t trow = t0 + 16 * w;
+
+    const uint2* src = reinterpret_cast<const uint2*>(x + trow * C + c0) + lane;
+    uint2 v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __ldg(src + (size_t)i * (size_t)(C >> 2));
+
+    float cm0 = 0.0f, cm1 = 0.0f, cm2 = 0.0f, cm3 = 0.0f, rm[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float a0 = fabsf(bf16_lo(v[i].x)), a1 = fabsf(bf16_hi(v[i].x));
+        const float a2 = fabsf(bf16_lo(v[i].y)), a3 = fabsf(bf16_hi(v[i].y));
+        cm0 = fmaxf(cm0, a0);
+        cm1 = fmaxf(cm1, a1);
+        cm2 = fmaxf(cm2, a2);
+        cm3 = fmaxf(cm3, a3);
+        rm[i] = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
+    }
+    *reinterpret_cast<float4*>(&red[w][4 * lane]) = make_float4(cm0, cm1, cm2, cm3);
+
+    // Row max-abs reduce-scatter: at the step with lane bit b, a lane keeps the half of its
+    // rows selected by that bit and sends the other half to its partner.
+    {
+        const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4, b1 = lane & 2;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float send = b4 ? rm[i] : rm[i + 8], keep = b4 ? rm[i + 8] : rm[i];
+            rm[i] = fmaxf(keep, __shfl_xor_sync(0xFFFFFFFFu, send, 16));
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float send = b3 ? rm[i] : rm[i + 4], keep = b3 ? rm[i + 4] : rm[i];
+            rm[i] = fmaxf(keep, __shfl_xor_sync(0xFFFFFFFFu, send, 8));
+        }
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const float send = b2 ? rm[i] : rm[i + 2], keep = b2 ? rm[i + 2] : rm[i];
+            rm[i] = fmaxf(keep, __shfl_xor_sync(0xFFFFFFFFu, send, 4));
+        }
+        {
+            const float send = b1 ? rm[0] : rm[1], keep = b1 ? rm[1] : rm[0];
+            rm[0] = fmaxf(keep, __shfl_xor_sync(0xFFFFFFFFu, send, 2));
+        }
+        rm[0] = fmaxf(rm[0], __shfl_xor_sync(0xFFFFFFFFu, rm[0], 1));
+    }
+    float rsc, rinv;
+    group_scale(rm[0], rsc, rinv);                      // row 16w + (lane >> 1)
+    if (!(lane & 1)) s[cb * T + trow + (lane >> 1)] = rsc;
+
+    __syncthreads();
+    if (threadIdx.x < 128) {
+        float a = red[0][threadIdx.x];
+#pragma unroll
+        for (int k = 1; k < 8; ++k) a = fmaxf(a, red[k][threadIdx.x]);
+        float sc, inv;
+        group_scale(a, sc, inv);
+        st[tb * C + c0 + threadIdx.x] = sc;
+        inv_c[threadIdx.x] = inv;
+    }
+
+    // Row-wise codes.
+    uint8_t* qrow = q + trow * C + c0 + 4 * lane;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float ri = __shfl_sync(0xFFFFFFFFu, rinv, 2 * i);
+        const uint32_t word =
+            e4m3x2(__fmul_rn(bf16_lo(v[i].x), ri), __fmul_rn(bf16_hi(v[i].x), ri)) |
+            (e4m3x2(__fmul_rn(bf16_lo(v[i].y), ri), __fmul_rn(bf16_hi(v[i].y), ri)) << 16);
+        *reinterpret_cast<uint32_t*>(qrow + (size_t)i * (size_t)C) = word;
+    }
+
+    __syncthreads();
+    const float4 ic = *reinterpret_cast<const float4*>(&inv_c[4 * lane]);
+    uint8_t* dst = qt + (c0 + 4 * lane) * T + trow;
+    uint32_t c[4][4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const uint2 a = v[4 * p], b = v[4 * p + 1], d = v[4 * p + 2], e = v[4 * p + 3];
+        c[0][p] = e4m3x2(__fmul_rn(bf16_lo(a.x), ic.x), __fmul_rn(bf16_lo(b.x), ic.x)) |
+                  (e4m3x2(__fmul_rn(bf16_lo(d.x), ic.x), __fmul_rn(bf16_lo(e.x), ic.x)) << 16);
+        c[1][p] = e4m3x2(__fmul_rn(bf16_hi(a.x), ic.y), __fmul_rn(bf16_hi(b.x), ic.y)) |
+                  (e4m3x2(__fmul_rn(bf16_hi(d.x), ic.y), __fmul_rn(bf16_hi(e.x), ic.y)) << 16);
+        c[2][p] = e4m3x2(__fmul_rn(bf16_lo(a.y), ic.z), __fmul_rn(bf16_lo(b.y), ic.z)) |
+                  (e4m3x2(__fmul_rn(bf16_lo(d.y), ic.z), __fmul_rn(bf16_lo(e.y), ic.z)) << 16);
+        c[3][p] = e4m3x2(__fmul_rn(bf16_hi(a.y), ic.w), __fmul_rn(bf16_hi(b.y), ic.w)) |
+                  (e4m3x2(__fmul_rn(bf16_hi(d.y), ic.w), __fmul_rn(bf16_hi(e.y), ic.w)) << 16);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        *reinterpret_cast<uint4*>(dst + (size_t)j * (size_t)T) = make_uint4(c[j][0], c[j][1], c[j][2], c[j][3]);
 }
 
 // ------------------------------------------------------------------------------------------

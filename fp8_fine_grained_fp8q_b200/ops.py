@@ -46,6 +46,7 @@ def lib() -> ctypes.CDLL:
     for name, args in {
         "fp8q_act_1x128": [P, I64, I64, P, P, P],
         "fp8q_act_128x1_transposed": [P, I64, I64, P, P, P],
+        "fp8q_act_dual": [P, I64, I64, P, P, P, P, P],
         "fp8q_weight_128x128": [P, I64, I64, P, P, P, P],
         "fp8_gemm_blockscaled": [I, P, P, P, P, P, I64, I64, I64, P, ctypes.c_size_t, P],
         "fp8_grouped_gemm_blockscaled": [P, P, P, P, P, I32, I64, I64, I64, P, P],
@@ -125,6 +126,21 @@ def act_128x1_transposed(x: torch.Tensor, qt: torch.Tensor | None = None,
     _check("fp8q_act_128x1_transposed",
            lib().fp8q_act_128x1_transposed(_p(x), T, C, _p(qt), _p(s), _stream(x.device)))
     return qt, s
+
+
+def act_dual(x: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tensor | None = None,
+             qt: torch.Tensor | None = None, st: torch.Tensor | None = None):
+    """x[T,C] bf16 -> (q[T,C], s[C/128, T], qt[C,T], st[T/128, C]) in one pass over x: the
+    outputs of act_1x128(x) and act_128x1_transposed(x), bit for bit."""
+    _require(x, "x", torch.bfloat16, 2)
+    T, C = x.shape
+    q = _out(q, (T, C), torch.uint8, x.device, "q")
+    s = _out(s, (C // 128, T), torch.float32, x.device, "s")
+    qt = _out(qt, (C, T), torch.uint8, x.device, "qt")
+    st = _out(st, (T // 128, C), torch.float32, x.device, "st")
+    _check("fp8q_act_dual",
+           lib().fp8q_act_dual(_p(x), T, C, _p(q), _p(s), _p(qt), _p(st), _stream(x.device)))
+    return q, s, qt, st
 
 
 def weight_128x128(w: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tensor | None = None,

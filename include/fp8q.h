@@ -107,6 +107,21 @@ FP8Q_API int fp8q_act_128x1_transposed(const uint16_t* x, int64_t T, int64_t C, 
                               fp8q_stream_t stream);
 
 /*
+ * Both activation forms of one tensor in a single pass over x: the 1x128 form (as
+ * fp8q_act_1x128 with M = T, K = C) and the 128x1 transposed form (as
+ * fp8q_act_128x1_transposed).  A linear layer needs both for X (Fprop, Wgrad) and for dY
+ * (Dgrad, Wgrad) ([REPOST] paragraphs 2 and 4); reading x once instead of twice saves one
+ * full read of the tensor from HBM.  Outputs are bit-identical to the two separate calls.
+ *   x : [T, C] bf16
+ *   q : [T, C] E4M3 codes,  s  : [C/128, T] fp32   (groups: one token, 128 channels)
+ *   qt: [C, T] E4M3 codes,  st : [T/128, C] fp32   (groups: one channel, 128 tokens)
+ * T % 128 == 0 and C % 128 == 0 (FP8Q_ERR_SHAPE otherwise); T / 128 <= 65535
+ * (FP8Q_ERR_UNSUPPORTED otherwise).  All pointers 16-byte aligned, caller-owned, device.
+ */
+FP8Q_API int fp8q_act_dual(const uint16_t* x, int64_t T, int64_t C, uint8_t* q, float* s,
+                           uint8_t* qt, float* st, fp8q_stream_t stream);
+
+/*
  * 128x128 block-wise weight quantisation ([SUMMARY] Key ideas, FP8 bullet).
  *   w : [N, K] bf16            q : [N, K] E4M3 codes         s : [N/128, K/128] fp32 scales
  *   qt_or_null : NULL, or [K, N] receiving the same codes transposed.

@@ -70,6 +70,18 @@ def test_act_128x1_host_checks(L):
     assert L.fp8q_act_128x1_transposed(P(FAKE), 128, 64, P(MISALIGNED), P(FAKE), s) == ERR_ALIGN
 
 
+def test_act_dual_host_checks(L):
+    s = None
+    d = L.fp8q_act_dual
+    assert d(P(FAKE), 128, 64, P(FAKE), P(FAKE), P(FAKE), P(FAKE), s) == ERR_SHAPE   # C % 128
+    assert d(P(FAKE), 100, 128, P(FAKE), P(FAKE), P(FAKE), P(FAKE), s) == ERR_SHAPE
+    assert d(P(FAKE), -128, 128, P(FAKE), P(FAKE), P(FAKE), P(FAKE), s) == ERR_ARG
+    assert d(P(FAKE), 0, 128, P(FAKE), P(FAKE), P(FAKE), P(FAKE), s) == OK
+    assert d(P(FAKE), 128, 128, P(FAKE), P(FAKE), None, P(FAKE), s) == ERR_ARG
+    assert d(P(FAKE), 128, 128, P(FAKE), P(FAKE), P(FAKE), P(MISALIGNED), s) == ERR_ALIGN
+    assert d(P(FAKE), 128 * 65536, 128, P(FAKE), P(FAKE), P(FAKE), P(FAKE), s) == ERR_UNSUPPORTED
+
+
 def test_weight_host_checks(L):
     s = None
     assert L.fp8q_weight_128x128(P(FAKE), 100, 128, P(FAKE), P(FAKE), None, s) == ERR_SHAPE

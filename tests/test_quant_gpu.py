@@ -127,6 +127,40 @@ def test_act_128x1_full_size(which):
     assert_same(gq, gs, oq, os_, f"128x1 {which}{bits.shape}")
 
 
+def run_dual(bits):
+    x = bf16_dev(bits)
+    T, C = bits.shape
+    q, s, qt, st = ops.act_dual(x, _poison_q((T, C)), _poison_s((C // 128, T)),
+                                _poison_q((C, T)), _poison_s((T // 128, C)))
+    torch.cuda.synchronize()
+    return host(q), host(s), host(qt), host(st)
+
+
+def check_dual(bits, what):
+    gq, gs, gqt, gst = run_dual(bits)
+    oq, os_ = oracle.quant_1x128(bits)
+    oqt, ost = oracle.quant_128x1_t(bits)
+    assert_same(gq, gs, oq, os_, f"dual 1x128 {what}")
+    assert_same(gqt, gst, oqt, ost, f"dual 128x1 {what}")
+
+
+@pytest.mark.parametrize("T,C", [(128, 128), (256, 384), (384, 1024)])
+def test_act_dual_small(T, C):
+    check_dual(synth.activations_channel_outliers(T, C, seed=T * 3 + C), f"{T}x{C}")
+
+
+def test_act_dual_special_values():
+    rows = special_values(256, 1024, seed=5)                 # specials in row groups
+    cols = special_values(1024, 256, seed=6).T.copy()        # specials in column groups
+    check_dual(np.concatenate([rows, cols], axis=0), "special")
+
+
+@pytest.mark.parametrize("which", ["X", "dY"])
+def test_act_dual_full_size(which):
+    bits = linear_layer_inputs()[which]
+    check_dual(bits, f"{which}{bits.shape}")
+
+
 def run_weight(bits, transposed):
     w = bf16_dev(bits)
     N, K = bits.shape
