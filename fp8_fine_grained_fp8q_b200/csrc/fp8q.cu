@@ -81,6 +81,21 @@ bool make_tmap_u8(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t ou
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Row-major output matrix [outer][inner] of 2- or 4-byte elements, stored by the GEMM epilogue in
+// boxes of 32 rows x 64 bytes with the 64-byte swizzle.
+bool make_tmap_out(CUtensorMap* tm, void* base, uint64_t inner, uint64_t outer, int elt_bytes)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {inner * (uint64_t)elt_bytes};
+    const cuuint32_t box[2] = {(cuuint32_t)(64 / elt_bytes), 32};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(tm, elt_bytes == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims,
+              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------------------------------------
 // GEMM launch
 // ------------------------------------------------------------------------------------------
@@ -153,6 +168,10 @@ int launch_gemm(const uint8_t* A, const float* sA, const uint8_t* B, const float
         const uint64_t rows = GROUPED ? (uint64_t)E * (uint64_t)N : (uint64_t)N;
         if (!make_tmap_u8(&tb, B, (uint64_t)K, rows, 128, BN)) return FP8Q_ERR_CUDA;
     }
+    CUtensorMap td;   // the epilogue's store map (the grouped GEMM stores without it)
+    memset(&td, 0, sizeof(td));
+    if (!GROUPED && !make_tmap_out(&td, D, (uint64_t)N, (uint64_t)M, MODE == kModeWgrad ? 4 : 2))
+        return FP8Q_ERR_CUDA;
     GemmArgs a;
     a.sA = sA;
     a.sB = sB;
@@ -191,7 +210,7 @@ int launch_gemm(const uint8_t* A, const float* sA, const uint8_t* B, const float
             attr[0].val.cooperative = 1;
             cfg.attrs = attr;
             cfg.numAttrs = 1;
-            if (cudaLaunchKernelEx(&cfg, gemm_blockscaled_kernel<MODE, BN, GROUPED>, ta, tb, a) != cudaSuccess) {
+            if (cudaLaunchKernelEx(&cfg, gemm_blockscaled_kernel<MODE, BN, GROUPED>, ta, tb, td, a) != cudaSuccess) {
                 cudaGetLastError();
                 return FP8Q_ERR_CUDA;
             }
@@ -200,7 +219,7 @@ int launch_gemm(const uint8_t* A, const float* sA, const uint8_t* B, const float
     }
     const int grid = (int)(tiles < sms ? tiles : sms);
     if (grid <= 0) return FP8Q_OK;
-    gemm_blockscaled_kernel<MODE, BN, GROUPED><<<grid, S::kThreads, S::kSmemBytes, st>>>(ta, tb, a);
+    gemm_blockscaled_kernel<MODE, BN, GROUPED><<<grid, S::kThreads, S::kSmemBytes, st>>>(ta, tb, td, a);
     return launch_status();
 }
 

@@ -112,7 +112,12 @@ struct GemmShape {
     static constexpr int kNumBars = 2 * kStages + 4 + 2 * kScaleStages + 2;
     static constexpr int kOffMisc = kOffBars + kNumBars * 8;
     static constexpr int kOffGroups = kOffMisc + 16;
-    static constexpr int kSmemBytes = kOffGroups + (GROUPED ? 2 * (kMaxGroups + 1) * 4 : 0) + 1024;
+    // Epilogue staging: 2 KB per promotion warp and buffer, 1024-byte aligned (the 64-byte
+    // swizzle of the tensor store works on absolute shared-memory address bits).  Two buffers per
+    // warp where shared memory allows, so one slab's store reads while the next is written.
+    static constexpr int kEpiBufs = (MODE == kModeWgrad || GROUPED) ? 1 : 2;
+    static constexpr int kOffEpi = (kOffGroups + (GROUPED ? 2 * (kMaxGroups + 1) * 4 : 0) + 1023) / 1024 * 1024;
+    static constexpr int kSmemBytes = kOffEpi + 8 * 2048 * kEpiBufs + 1024;
     // Registers: launched at 168 per thread (384 x 168 = 64512); 128 x 40 + 256 x 232 = 64512.
     static constexpr int kRegsLow = 40;
     static constexpr int kRegsHigh = 232;
@@ -162,7 +167,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 template <int MODE, int BN, bool GROUPED>
 __global__ void __launch_bounds__(384, 1)
 gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                        const GemmArgs args)
+                        const __grid_constant__ CUtensorMap tmD, const GemmArgs args)
 {
     using S = GemmShape<MODE, BN, GROUPED>;
     extern __shared__ uint8_t smem_raw[];
@@ -354,9 +359,10 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
         const int ptid = pw * 32 + lane;      // promotion thread 0..255
         int tb = 0, ss = 0;
         uint32_t tph = 0, sph = 0;
-        // Columns per TMEM load: 16 at BN = 256 (two chunks in flight still fit beside the 128
-        // accumulators), 32 at BN = 128.
-        constexpr int kCW = 16;
+        // Columns per TMEM load.  Each load is a round trip on the promotion's critical path,
+        // so chunks are as wide as the registers allow: two 32-column chunks in flight beside
+        // the BN/2 accumulators; 16 for Wgrad, whose chunks also carry their column scales.
+        constexpr int kCW = (MODE == kModeWgrad || S::kHalf < 32) ? 16 : 32;
         constexpr int kChunks = S::kHalf / kCW;
         float2 acc[S::kHalf / 2];
         WorkSched wsched = sched_begin(args);
@@ -494,28 +500,73 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                 }
                 if (!alive) break;
             }
-            // Epilogue: rows of this tile's group only.
-            if (row < ti.row_end) {
-                if (MODE == kModeWgrad) {
-                    float* drow = reinterpret_cast<float*>(args.D) + (size_t)row * args.N + ncol0;
+            // Epilogue.  The warp's 32 rows x BN/2 columns leave through 2 KB staging buffers in
+            // shared memory, one 32-row x 64-byte slab at a time.  16-byte unit p of staged row r
+            // sits at unit 4r + (p ^ ((r >> 1) & 3)) -- the tensor map's 64-byte swizzle, and
+            // conflict-free for the row-per-lane writes.  Dense GEMMs hand each slab to a bulk
+            // tensor store (rows past M are clipped by the tensor bounds); the grouped GEMM,
+            // whose next rows belong to another group, stores the slab itself, 8 rows x 64
+            // contiguous bytes per instruction, skipping rows at or past the group's end.
+            {
+                constexpr int kElt = (MODE == kModeWgrad) ? 4 : 2;    // bytes per output element
+                constexpr int kSlabCols = 64 / kElt;
+                uint4* stage0 = reinterpret_cast<uint4*>(smem + S::kOffEpi) + pw * 128 * S::kEpiBufs;
+                const int wrow0 = ti.row0 + quad * 32;
 #pragma unroll
-                    for (int j = 0; j < S::kHalf / 2; j += 2)
-                        *reinterpret_cast<float4*>(drow + 2 * j) =
-                            make_float4(acc[j].x, acc[j].y, acc[j + 1].x, acc[j + 1].y);
-                } else {
-                    uint16_t* drow = reinterpret_cast<uint16_t*>(args.D) + (size_t)row * args.N + ncol0;
+                for (int sl = 0; sl < S::kHalf / kSlabCols; ++sl) {
+                    uint4* stage = stage0 + (sl % S::kEpiBufs) * 128;
+                    uint4 u[4];
 #pragma unroll
-                    for (int j = 0; j < S::kHalf / 2; j += 4) {
-                        uint4 o;
-                        o.x = pack_bf16x2(acc[j + 0].x, acc[j + 0].y);
-                        o.y = pack_bf16x2(acc[j + 1].x, acc[j + 1].y);
-                        o.z = pack_bf16x2(acc[j + 2].x, acc[j + 2].y);
-                        o.w = pack_bf16x2(acc[j + 3].x, acc[j + 3].y);
-                        *reinterpret_cast<uint4*>(drow + 2 * j) = o;
+                    for (int p = 0; p < 4; ++p) {
+                        if (MODE == kModeWgrad) {
+                            const float2 a = acc[sl * 8 + 2 * p], b = acc[sl * 8 + 2 * p + 1];
+                            u[p] = make_uint4(__float_as_uint(a.x), __float_as_uint(a.y), __float_as_uint(b.x),
+                                              __float_as_uint(b.y));
+                        } else {
+                            const int q = sl * 16 + 4 * p;
+                            u[p] = make_uint4(pack_bf16x2(acc[q].x, acc[q].y), pack_bf16x2(acc[q + 1].x, acc[q + 1].y),
+                                              pack_bf16x2(acc[q + 2].x, acc[q + 2].y),
+                                              pack_bf16x2(acc[q + 3].x, acc[q + 3].y));
+                        }
+                    }
+                    if (!GROUPED) {
+                        // The buffer is free once the store issued from it kEpiBufs slabs ago has
+                        // read it.
+                        if (lane == 0) bulk_wait_group_read<S::kEpiBufs - 1>();
+                        __syncwarp();
+                    }
+                    const int wsw = (lane >> 1) & 3;
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) stage[lane * 4 + (p ^ wsw)] = u[p];
+                    if (!GROUPED) {
+                        fence_proxy_async_smem();     // the writes above, before the async-proxy read
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&tmD, smem_u32(stage), ncol0 + sl * kSlabCols, wrow0);
+                            bulk_commit_group();
+                        }
+                    } else {
+                        __syncwarp();
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int r = (lane >> 2) + 8 * i, p = lane & 3;
+                            const uint4 v = stage[r * 4 + (p ^ ((r >> 1) & 3))];
+                            const int grow = wrow0 + r;
+                            if (grow < ti.row_end) {
+                                uint8_t* dst = reinterpret_cast<uint8_t*>(args.D) +
+                                               ((size_t)grow * args.N + ncol0 + sl * kSlabCols) * kElt + p * 16;
+                                *reinterpret_cast<uint4*>(dst) = v;
+                            }
+                        }
+                        __syncwarp();
                     }
                 }
             }
         }
+        // Every store has finished reading shared memory and writing its tile before the CTA
+        // (and its shared memory) goes away.
+        if (!GROUPED && lane == 0) bulk_wait_group<0>();
+        __syncwarp();
         tc_fence_before();
         named_bar_arrive(1, 32 + 256);
     }
