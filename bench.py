@@ -56,10 +56,13 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def source_hash() -> str:
+GEMM_SOURCES = ("gemm.cuh", "ptx.cuh")         # what the GEMM kernel's DRAM traffic depends on
+
+
+def source_hash(names=GEMM_SOURCES) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "fp8_fine_grained_fp8q_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted(names):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
@@ -67,7 +70,8 @@ def source_hash() -> str:
 
 
 def load_traffic():
-    """DRAM bytes per launch from the committed ncu summary, if taken on this source."""
+    """DRAM bytes per GEMM launch from the committed ncu summary, if it was taken on the GEMM
+    sources as they are now (else None: the counters describe another kernel)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
@@ -90,7 +94,7 @@ class ClockSampler:
         0x100: "display_clock_setting",
     }
 
-    def __init__(self, device_index: int, period_s: float = 0.02):
+    def __init__(self, device_index: int, period_s: float = 0.002):
         self.samples = []
         self.reasons = set()
         self.max_mhz = None

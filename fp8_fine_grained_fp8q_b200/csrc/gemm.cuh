@@ -385,6 +385,13 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
             }
 #pragma unroll
             for (int i = 0; i < S::kHalf / 2; ++i) acc[i] = make_float2(0.0f, 0.0f);
+            // The row and block scales of the item's groups are pulled into L2 up front (one line
+            // per group holds this warp's 32 row scales), so the per-group loads below, issued one
+            // group ahead, find them there instead of in HBM.
+            for (int k = it.kb0 + 1 + lane; k < it.kb1; k += 32) {
+                prefetch_l2(args.sA + (size_t)k * args.M + min(ti.row0 + quad * 32, args.M - 1));
+                if (MODE != kModeWgrad) prefetch_l2(sb_ptr + (size_t)k * sb_step);
+            }
             float sa_next = in_a ? __ldg(sa_ptr + (size_t)it.kb0 * args.M) : 0.0f;
             float sb_next = (MODE != kModeWgrad) ? __ldg(sb_ptr + (size_t)it.kb0 * sb_step) : 1.0f;
             bool ok = true;

@@ -154,6 +154,9 @@ __device__ __forceinline__ void named_bar_arrive(uint32_t id, uint32_t count)
 // ------------------------------------------------------------------------------------------
 // TMA
 // ------------------------------------------------------------------------------------------
+// Fetch the line holding p into L2 (no register result, nothing waits on it).
+__device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* tm)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"(tm) : "memory");
