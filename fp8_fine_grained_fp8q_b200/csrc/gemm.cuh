@@ -361,9 +361,18 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
         uint32_t tph = 0, sph = 0;
         // Columns per TMEM load.  Each load is a round trip on the promotion's critical path,
         // so chunks are as wide as the registers allow: two 32-column chunks in flight beside
-        // the BN/2 accumulators; 16 for Wgrad, whose chunks also carry their column scales.
+        // the BN/2 accumulators.
+        //
+        // Wgrad multiplies every element by its own column's scale, which comes from shared
+        // memory; with one row per thread each thread would need all BN/2 column scales per K
+        // group.  So Wgrad reads TMEM with the 16x256b shape instead: a thread holds 4 rows
+        // (t/4 + 8i of the warp's 32) x 2 columns of every 8-column block, i.e. needs a quarter
+        // of the column scales (an 8-byte load per block).  Its chunk is 16 columns (16
+        // registers); acc[kBlocks * i + j] is row i's column pair of block j.
         constexpr int kCW = (MODE == kModeWgrad || S::kHalf < 32) ? 16 : 32;
         constexpr int kChunks = S::kHalf / kCW;
+        constexpr int kBlocks = S::kHalf / 8;
+        const int wt0 = lane & 3, wt1 = lane >> 2;   // Wgrad: column pair and first row of a thread
         float2 acc[S::kHalf / 2];
         WorkSched wsched = sched_begin(args);
         WorkItem it;
@@ -409,12 +418,28 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                 const uint32_t taddr = tmem_base + lane_base + (uint32_t)(tb * BN + half * S::kHalf);
                 const float* cs = col_scales + ss * BN + half * S::kHalf;
                 const float2 c2 = make_float2(sa * sbv, sa * sbv);
-                const float2 sa2 = make_float2(sa, sa);
+                // Wgrad: the row scales of this thread's 4 rows, from the lanes that loaded them.
+                float2 sa2w[4];
+                if (MODE == kModeWgrad) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float v = __shfl_sync(0xFFFFFFFFu, sa, wt1 + 8 * i);
+                        sa2w[i] = make_float2(v, v);
+                    }
+                }
+                const auto tload = [&](int ch, uint32_t (&r)[kCW]) {
+                    if (MODE != kModeWgrad) {
+                        tmem_ld_async(taddr + ch * kCW, r);
+                    } else {
+                        tmem_ld_16x256b_x2(taddr + ch * kCW, r);
+                        tmem_ld_16x256b_x2(taddr + (16u << 16) + ch * kCW, r + 8);
+                    }
+                };
                 // Two register chunks: the TMEM load of chunk ch+1 is in flight while chunk ch is
                 // folded into the accumulators.  The buffer is released as soon as its last
                 // chunk has landed in registers, before that chunk's arithmetic.
                 uint32_t ra[kCW], rb[kCW];
-                tmem_ld_async(taddr, ra);
+                tload(0, ra);
                 tmem_wait_ld(ra);
                 const auto fold = [&](uint32_t (&cur)[kCW], int ch) {
                     if (MODE != kModeWgrad) {
@@ -424,15 +449,20 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                             acc[(ch * kCW + j) / 2] = __ffma2_rn(v, c2, acc[(ch * kCW + j) / 2]);
                         }
                     } else {
+                        // cur[8h + 4b + 2q + {0,1}]: row wt1 + 8q + 16h, column pair of block 2ch + b.
 #pragma unroll
-                        for (int j = 0; j < kCW; j += 4) {
-                            const float4 c4 = *reinterpret_cast<const float4*>(cs + ch * kCW + j);
-                            const float2 s01 = __fmul2_rn(sa2, make_float2(c4.x, c4.y));
-                            const float2 s23 = __fmul2_rn(sa2, make_float2(c4.z, c4.w));
-                            const float2 v01 = make_float2(__uint_as_float(cur[j]), __uint_as_float(cur[j + 1]));
-                            const float2 v23 = make_float2(__uint_as_float(cur[j + 2]), __uint_as_float(cur[j + 3]));
-                            acc[(ch * kCW + j) / 2] = __ffma2_rn(v01, s01, acc[(ch * kCW + j) / 2]);
-                            acc[(ch * kCW + j) / 2 + 1] = __ffma2_rn(v23, s23, acc[(ch * kCW + j) / 2 + 1]);
+                        for (int b = 0; b < 2; ++b) {
+                            const int jb = 2 * ch + b;
+                            const float2 sc = *reinterpret_cast<const float2*>(cs + 8 * jb + 2 * wt0);
+#pragma unroll
+                            for (int h = 0; h < 2; ++h) {
+#pragma unroll
+                                for (int q = 0; q < 2; ++q) {
+                                    const int i = 2 * h + q, r0 = 8 * h + 4 * b + 2 * q;
+                                    const float2 v = make_float2(__uint_as_float(cur[r0]), __uint_as_float(cur[r0 + 1]));
+                                    acc[kBlocks * i + jb] = __ffma2_rn(v, __fmul2_rn(sa2w[i], sc), acc[kBlocks * i + jb]);
+                                }
+                            }
                         }
                     }
                 };
@@ -444,8 +474,8 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
 #pragma unroll
                 for (int ch = 0; ch < kChunks; ++ch) {
                     if (ch + 1 < kChunks) {
-                        if (ch & 1) tmem_ld_async(taddr + (ch + 1) * kCW, ra);
-                        else tmem_ld_async(taddr + (ch + 1) * kCW, rb);
+                        if (ch & 1) tload(ch + 1, ra);
+                        else tload(ch + 1, rb);
                     } else {
                         release();
                     }
@@ -526,9 +556,7 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
 #pragma unroll
                     for (int p = 0; p < 4; ++p) {
                         if (MODE == kModeWgrad) {
-                            const float2 a = acc[sl * 8 + 2 * p], b = acc[sl * 8 + 2 * p + 1];
-                            u[p] = make_uint4(__float_as_uint(a.x), __float_as_uint(a.y), __float_as_uint(b.x),
-                                              __float_as_uint(b.y));
+                            u[p] = make_uint4(0u, 0u, 0u, 0u);   // Wgrad stages 8-byte pieces below
                         } else {
                             const int q = sl * 16 + 4 * p;
                             u[p] = make_uint4(pack_bf16x2(acc[q].x, acc[q].y), pack_bf16x2(acc[q + 1].x, acc[q + 1].y),
@@ -542,9 +570,24 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                         if (lane == 0) bulk_wait_group_read<S::kEpiBufs - 1>();
                         __syncwarp();
                     }
-                    const int wsw = (lane >> 1) & 3;
+                    if (MODE == kModeWgrad) {
+                        // Slab sl = blocks 2sl, 2sl+1 (16 fp32 columns).  This thread's pair of block
+                        // 2sl + b in row r = wt1 + 8i is bytes 32b + 8*wt0 of the 64-byte staged row.
+                        float2* st2 = reinterpret_cast<float2*>(stage);
 #pragma unroll
-                    for (int p = 0; p < 4; ++p) stage[lane * 4 + (p ^ wsw)] = u[p];
+                        for (int i = 0; i < 4; ++i) {
+                            const int r = wt1 + 8 * i;
+#pragma unroll
+                            for (int b = 0; b < 2; ++b) {
+                                const int unit = (2 * b + (wt0 >> 1)) ^ ((r >> 1) & 3);
+                                st2[r * 8 + unit * 2 + (wt0 & 1)] = acc[kBlocks * i + 2 * sl + b];
+                            }
+                        }
+                    } else {
+                        const int wsw = (lane >> 1) & 3;
+#pragma unroll
+                        for (int p = 0; p < 4; ++p) stage[lane * 4 + (p ^ wsw)] = u[p];
+                    }
                     if (!GROUPED) {
                         fence_proxy_async_smem();     // the writes above, before the async-proxy read
                         __syncwarp();

@@ -328,6 +328,19 @@ __device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[16])
                  : "memory");
 }
 
+// 16 TMEM lanes x 2 blocks of 8 columns, starting at taddr's lane and column.  Thread t receives
+// lanes (t/4, t/4 + 8) x columns (2(t%4), 2(t%4) + 1) of each block:
+//   r[4j + 0], r[4j + 1]: lane t/4,     block j;   r[4j + 2], r[4j + 3]: lane t/4 + 8, block j.
+// Asynchronous like tmem_ld16_async: complete it with tmem_wait_ld.
+__device__ __forceinline__ void tmem_ld_16x256b_x2(uint32_t taddr, uint32_t* r)
+{
+    asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                   "=r"(r[7])
+                 : "r"(taddr)
+                 : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld_async(uint32_t taddr, uint32_t (&r)[16]) { tmem_ld16_async(taddr, r); }
 __device__ __forceinline__ void tmem_ld_async(uint32_t taddr, uint32_t (&r)[32]) { tmem_ld32_async(taddr, r); }
 
