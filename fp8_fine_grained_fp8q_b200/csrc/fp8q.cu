@@ -43,6 +43,54 @@ int launch_status()
     return e == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
+// Launches: every kernel of this library waits (griddepcontrol.wait) for the previous kernel in
+// the stream before touching global memory, so each may be launched with programmatic stream
+// serialization: its launch and prologue then overlap the previous kernel's tail.
+// FP8Q_PDL=0 turns this off (plain stream order).
+bool pdl_enabled()
+{
+    static const bool on = [] {
+        const char* e = getenv("FP8Q_PDL");
+        return !(e && strcmp(e, "0") == 0);
+    }();
+    return on;
+}
+
+template <typename... KArgs, typename... Args>
+int launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool cooperative,
+                  Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    int n = 0;
+    if (cooperative) {
+        attr[n].id = cudaLaunchAttributeCooperative;
+        attr[n].val.cooperative = 1;
+        ++n;
+    }
+    const int n_base = n;
+    if (pdl_enabled()) {
+        attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[n].val.programmaticStreamSerializationAllowed = 1;
+        ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    if (cudaLaunchKernelEx(&cfg, kern, args...) == cudaSuccess) return launch_status();
+    cudaGetLastError();
+    if (n == n_base) return FP8Q_ERR_CUDA;
+    cfg.numAttrs = n_base;   // the driver refused the combination: launch in plain stream order
+    if (cudaLaunchKernelEx(&cfg, kern, args...) != cudaSuccess) {
+        cudaGetLastError();
+        return FP8Q_ERR_CUDA;
+    }
+    return launch_status();
+}
+
 // ------------------------------------------------------------------------------------------
 // TMA descriptors (the driver entry point is fetched through the runtime, so the library has
 // no link-time dependency on libcuda).
@@ -200,27 +248,14 @@ int launch_gemm(const uint8_t* A, const float* sA, const uint8_t* B, const float
             a.stamp = next_stamp();
             a.units = units;
             // CTAs wait on each other's partials: launch them co-resident (cooperative launch).
-            cudaLaunchConfig_t cfg = {};
-            cfg.gridDim = dim3((unsigned)grid);
-            cfg.blockDim = dim3(S::kThreads);
-            cfg.dynamicSmemBytes = S::kSmemBytes;
-            cfg.stream = st;
-            cudaLaunchAttribute attr[1];
-            attr[0].id = cudaLaunchAttributeCooperative;
-            attr[0].val.cooperative = 1;
-            cfg.attrs = attr;
-            cfg.numAttrs = 1;
-            if (cudaLaunchKernelEx(&cfg, gemm_blockscaled_kernel<MODE, BN, GROUPED>, ta, tb, td, a) != cudaSuccess) {
-                cudaGetLastError();
-                return FP8Q_ERR_CUDA;
-            }
-            return launch_status();
+            return launch_kernel(gemm_blockscaled_kernel<MODE, BN, GROUPED>, dim3((unsigned)grid),
+                                 dim3(S::kThreads), S::kSmemBytes, st, true, ta, tb, td, a);
         }
     }
     const int grid = (int)(tiles < sms ? tiles : sms);
     if (grid <= 0) return FP8Q_OK;
-    gemm_blockscaled_kernel<MODE, BN, GROUPED><<<grid, S::kThreads, S::kSmemBytes, st>>>(ta, tb, td, a);
-    return launch_status();
+    return launch_kernel(gemm_blockscaled_kernel<MODE, BN, GROUPED>, dim3((unsigned)grid), dim3(S::kThreads),
+                         S::kSmemBytes, st, false, ta, tb, td, a);
 }
 
 // Tile width: 256 whenever N allows it (measured faster on every linear-layer and MLA shape: it
@@ -330,8 +365,8 @@ int fp8q_act_1x128(const uint16_t* x, int64_t M, int64_t K, uint8_t* q, float* s
     const int64_t want = (ntiles + 32 * kUnr - 1) / (32 * kUnr);   // blocks of 32 eight-lane groups
     const int64_t cap = (int64_t)sms * 8;
     const int grid = (int)(want < cap ? want : cap);
-    act_1x128_kernel<kUnr><<<grid, 256, 0, (cudaStream_t)stream>>>(x, q, s, (int)M, (int)K);
-    return launch_status();
+    return launch_kernel(act_1x128_kernel<kUnr>, dim3(grid), dim3(256), 0, (cudaStream_t)stream, false, x, q, s,
+                         (int)M, (int)K);
 }
 
 int fp8q_act_128x1_transposed(const uint16_t* x, int64_t T, int64_t C, uint8_t* qt, float* s,
@@ -344,8 +379,7 @@ int fp8q_act_128x1_transposed(const uint16_t* x, int64_t T, int64_t C, uint8_t* 
     if (!aligned16(x) || !aligned16(qt) || !aligned16(s)) return FP8Q_ERR_ALIGN;
     if (T / 128 > 65535 || C / 64 > 0x7FFFFFFF) return FP8Q_ERR_UNSUPPORTED;
     const dim3 grid((unsigned)(C / 64), (unsigned)(T / 128));
-    act_128x1_t_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(x, qt, s, T, C);
-    return launch_status();
+    return launch_kernel(act_128x1_t_kernel, grid, dim3(256), 0, (cudaStream_t)stream, false, x, qt, s, T, C);
 }
 
 int fp8q_act_dual(const uint16_t* x, int64_t T, int64_t C, uint8_t* q, float* s, uint8_t* qt, float* st,
@@ -359,8 +393,7 @@ int fp8q_act_dual(const uint16_t* x, int64_t T, int64_t C, uint8_t* q, float* s,
         return FP8Q_ERR_ALIGN;
     if (T / 128 > 65535 || C / 128 > 0x7FFFFFFF) return FP8Q_ERR_UNSUPPORTED;
     const dim3 grid((unsigned)(C / 128), (unsigned)(T / 128));
-    act_dual_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(x, q, s, qt, st, T, C);
-    return launch_status();
+    return launch_kernel(act_dual_kernel, grid, dim3(256), 0, (cudaStream_t)stream, false, x, q, s, qt, st, T, C);
 }
 
 int fp8q_weight_128x128(const uint16_t* w, int64_t N, int64_t K, uint8_t* q, float* s, uint8_t* qt_or_null,
@@ -373,8 +406,8 @@ int fp8q_weight_128x128(const uint16_t* w, int64_t N, int64_t K, uint8_t* q, flo
     if (!aligned16(w) || !aligned16(q) || !aligned16(s) || !aligned16(qt_or_null)) return FP8Q_ERR_ALIGN;
     if (N / 128 > 65535 || K / 128 > 0x7FFFFFFF) return FP8Q_ERR_UNSUPPORTED;
     const dim3 grid((unsigned)(K / 128), (unsigned)(N / 128));
-    weight_128x128_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(w, q, s, qt_or_null, N, K);
-    return launch_status();
+    return launch_kernel(weight_128x128_kernel, grid, dim3(256), 0, (cudaStream_t)stream, false, w, q, s, qt_or_null,
+                         N, K);
 }
 
 size_t fp8q_gemm_workspace_size(int mode, int64_t M, int64_t N, int64_t K)

@@ -190,6 +190,7 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    griddep_launch_dependents();
 
     // ---------------------------------------------------------------- set-up
     if (threadIdx.x == 0) {
@@ -219,6 +220,8 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
         tmem_alloc(smem_u32(misc), S::kTmemCols);
         tmem_relinquish();
     }
+    // Everything above touches only this CTA's own resources; inputs are read from here on.
+    griddep_wait();
     if (GROUPED && warp == 2) {
         // Copy the offsets, validate them and build the prefix of 128-row tiles per group with a
         // warp scan (each lane owns a contiguous run of groups).

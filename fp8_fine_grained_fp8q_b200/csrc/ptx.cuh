@@ -154,6 +154,14 @@ __device__ __forceinline__ void named_bar_arrive(uint32_t id, uint32_t count)
 // ------------------------------------------------------------------------------------------
 // TMA
 // ------------------------------------------------------------------------------------------
+// Programmatic dependent launch.  A kernel launched with programmatic stream serialization may
+// start while the previous kernel in the stream is finishing; griddep_wait() blocks until that
+// kernel has completed and its memory is visible, so every kernel here calls it before its first
+// global-memory access.  griddep_launch_dependents() lets the next kernel in the stream start its
+// own launch (and its pre-wait prologue) early.  Both are no-ops for a normal launch.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Fetch the line holding p into L2 (no register result, nothing waits on it).
 __device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
 

@@ -12,6 +12,8 @@
 
 #include <stdint.h>
 
+#include "ptx.cuh"
+
 namespace fp8q {
 
 constexpr float kE4M3Max = 448.0f;
@@ -76,6 +78,8 @@ __global__ void __launch_bounds__(256) act_1x128_kernel(const uint16_t* __restri
                                                         uint8_t* __restrict__ q,
                                                         float* __restrict__ s, int M, int K)
 {
+    griddep_launch_dependents();
+    griddep_wait();
     const uint32_t KB = (uint32_t)K >> 7;
     const uint32_t ntiles = (uint32_t)M * KB;
     const uint32_t sub = threadIdx.x & 7;                       // lane within the tile
@@ -133,6 +137,8 @@ __global__ void __launch_bounds__(256) act_128x1_t_kernel(const uint16_t* __rest
                                                           uint8_t* __restrict__ qt,
                                                           float* __restrict__ s, int64_t T, int64_t C)
 {
+    griddep_launch_dependents();
+    griddep_wait();
     __shared__ float red[8][kT1Ch];
     __shared__ float inv_c[kT1Ch];
 
@@ -194,6 +200,8 @@ __global__ void __launch_bounds__(256, 3) act_dual_kernel(const uint16_t* __rest
                                                        uint8_t* __restrict__ qt, float* __restrict__ st,
                                                        int64_t T, int64_t C)
 {
+    griddep_launch_dependents();
+    griddep_wait();
     __shared__ __align__(16) float red[8][128];
     __shared__ __align__(16) float inv_c[128];
 
@@ -301,6 +309,8 @@ __global__ void __launch_bounds__(256) weight_128x128_kernel(const uint16_t* __r
                                                              float* __restrict__ s,
                                                              uint8_t* __restrict__ qt, int64_t N, int64_t K)
 {
+    griddep_launch_dependents();
+    griddep_wait();
     __shared__ float red[8];
     __shared__ __align__(16) uint8_t codes[128][128 + 16];
 
