@@ -446,6 +446,124 @@ def run_reference(args, rank, world):
     }
 
 
+# ------------------------------------------------------------------------------------------ #
+# Secondary workload: the grouped MoE Fprop (--workload moe)
+# ------------------------------------------------------------------------------------------ #
+MOE_TOKENS, MOE_E, MOE_TOPK, MOE_N, MOE_K = 8192, 256, 8, 2048, 7168
+MOE_WORKLOAD = ("grouped MoE Fprop: 8192 tokens x top-8 of 256 experts (Zipf(1.1)-skewed, 8 empty), "
+                "act 1x128 of the expert-ordered rows [65536, 7168] + weight 128x128 of all experts "
+                "[256 x 2048, 7168] + ragged grouped GEMM")
+
+
+def run_moe(args, rank, world, dist):
+    """One step = 1x128 quantisation of the expert-ordered activations, 128x128 quantisation of all
+    expert weights, and the grouped GEMM; value = grouped-GEMM FLOPs / step time.  Inputs are
+    generated on the device (seeded): X ~ N(0,1) with 7 outlier channels x100, W_e ~ N(0, 0.02)."""
+    import torch
+    from fp8_fine_grained_fp8q_b200 import ops, synth
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ops.lib()
+    expert_of, counts = synth.moe_routing(tokens=MOE_TOKENS, experts=MOE_E, top_k=MOE_TOPK)
+    token_idx, off = synth.moe_grouped_rows(expert_of, MOE_E)
+    mtot = int(off[-1])
+    g = torch.Generator(device=dev)
+    g.manual_seed(synth.SEED_BASE + 5)
+    x = torch.randn((MOE_TOKENS, MOE_K), device=dev, generator=g)
+    outl = torch.randperm(MOE_K, device=dev, generator=g)[: round(0.001 * MOE_K)]
+    x[:, outl] *= 100.0
+    xg = x.to(torch.bfloat16)[torch.from_numpy(token_idx).to(dev)].contiguous()
+    del x
+    w = torch.empty((MOE_E * MOE_N, MOE_K), dtype=torch.bfloat16, device=dev)
+    for e0 in range(0, MOE_E, 32):
+        w[e0 * MOE_N:(e0 + 32) * MOE_N] = (0.02 * torch.randn((32 * MOE_N, MOE_K), device=dev, generator=g)).to(torch.bfloat16)
+    offsets = torch.from_numpy(off).to(dev)
+    xq = torch.empty((mtot, MOE_K), dtype=torch.uint8, device=dev)
+    sx = torch.empty((MOE_K // 128, mtot), dtype=torch.float32, device=dev)
+    wq = torch.empty((MOE_E * MOE_N, MOE_K), dtype=torch.uint8, device=dev)
+    sw = torch.empty((MOE_E * MOE_N // 128, MOE_K // 128), dtype=torch.float32, device=dev)
+    out = torch.empty((mtot, MOE_N), dtype=torch.bfloat16, device=dev)
+    names = ["act_1x128_X", "weight_128x128_W", "grouped_gemm"]
+    launches = [
+        lambda: ops.act_1x128(xg, xq, sx),
+        lambda: ops.weight_128x128(w, wq, sw),
+        lambda: ops.grouped_gemm_blockscaled(xq, sx, wq.view(MOE_E, MOE_N, MOE_K),
+                                             sw.view(MOE_E, MOE_N // 128, MOE_K // 128), offsets, out),
+    ]
+    flop = 2.0 * mtot * MOE_N * MOE_K
+    work = {"act_1x128_X": ("bytes", mtot * MOE_K * QB_1x128),
+            "weight_128x128_W": ("bytes", MOE_E * MOE_N * MOE_K * QB_128x128),
+            "grouped_gemm": ("flop", flop)}
+    flush_w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+
+    def flush_l2():
+        flush_w.zero_()
+        flush_r.sum()
+
+    for _ in range(args.warmup):
+        flush_l2()
+        for f in launches:
+            f()
+    torch.cuda.synchronize()
+    if ops.device_status(dev) != ops.DEV_OK:
+        raise RuntimeError("device status after warm-up")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    with ClockSampler(local) as clocks:
+        for s_ in range(args.steps):
+            flush_l2()
+            evs[s_][0].record()
+            for f in launches:
+                f()
+            evs[s_][1].record()
+        torch.cuda.synchronize()
+    if ops.device_status(dev) != ops.DEV_OK:
+        raise RuntimeError("device status in the timed region")
+    ms_per_step = statistics.mean(e0.elapsed_time(e1) for e0, e1 in evs)
+    bsteps = min(args.steps, 10)
+    bevs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(launches) + 1)] for _ in range(bsteps)]
+    for s_ in range(bsteps):
+        flush_l2()
+        bevs[s_][0].record()
+        for i, f in enumerate(launches):
+            f()
+            bevs[s_][i + 1].record()
+    torch.cuda.synchronize()
+    peaks, peak_kind = load_peaks()
+    fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
+    kernels = {}
+    for i, name in enumerate(names):
+        ms = statistics.mean(b[i].elapsed_time(b[i + 1]) for b in bevs)
+        kind, amount = work[name]
+        if kind == "flop":
+            ach = amount / (ms * 1e-3) / 1e12
+            kernels[name] = {"ms": round(ms, 4), "TFLOP/s": round(ach, 1), "frac_fp8_peak": round(ach / fp8_peak, 4)}
+        else:
+            ach = amount / (ms * 1e-3) / 1e9
+            kernels[name] = {"ms": round(ms, 4), "GB/s": round(ach, 1), "frac_hbm": round(ach / peaks["hbm_gbs"], 4)}
+    g_ms = kernels["grouped_gemm"]["ms"]
+    return {
+        "metric": METRIC, "value": round(world * flop / (ms_per_step * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8_e4m3 (fp32 accumulate)", "data": "synthetic (seeded, generated on the device)",
+        "config": {"workload": MOE_WORKLOAD, "rows": mtot, "experts": MOE_E,
+                   "empty_experts": int((counts == 0).sum()), "max_rows": int(counts.max()),
+                   "n": MOE_N, "k": MOE_K, "l2": "flushed before every step (256 MiB write, then read)"},
+        "roofline": {"kernel": "gemm_blockscaled_kernel (grouped)", "bound": "tensor",
+                     "achieved": round(flop / (g_ms * 1e-3) / 1e12, 1), "peak": round(fp8_peak, 1),
+                     "unit": "TFLOP/s", "frac": round(flop / (g_ms * 1e-3) / 1e12 / fp8_peak, 4),
+                     "peak_source": f"{peak_kind} bf16 burst x {FP8_OVER_BF16}", "traffic": None},
+        "kernels": kernels,
+        "e2e": None,
+        "e2e_note": "not measured for this secondary workload (the expert weights alone are 7.5 GB of H2D per step)",
+        "gpu_launches": len(launches) * args.steps,
+        "clocks": clocks.summary(),
+    }
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -454,6 +572,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle CPU work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=["linear", "moe"], default="linear",
+                    help="linear: the FP8 linear layer (the headline); moe: the grouped MoE Fprop")
     ap.add_argument("--separate-quant", action="store_true",
                     help="quantise X and dY with separate 1x128 and 128x1 launches")
     args = ap.parse_args()
@@ -478,7 +598,7 @@ def main():
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         dist = tdist
     try:
-        line = run_ours(args, rank, world, dist)
+        line = (run_moe if args.workload == "moe" else run_ours)(args, rank, world, dist)
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:

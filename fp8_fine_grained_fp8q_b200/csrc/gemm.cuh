@@ -10,14 +10,18 @@
 // Here the overlap comes from the asynchronous tcgen05 pipeline instead:
 //   warp 0      TMA producer: A and B tiles (128-byte swizzled) into a STAGES-deep ring;
 //               for Wgrad also the per-column scales of each K group (bulk copy).
-//   warp 1      MMA issuer: 4 x tcgen05.mma (K = 32 each) per K group into one of two TMEM
-//               partial buffers (a fresh accumulation per group), then tcgen05.commit.
-//   warps 4-11  promotion: tcgen05.ld the partial of group kb while the tensor cores fill the
-//               other buffer, fold in the scales and accumulate in registers (each warp owns 32
-//               rows x BN/2 columns); after the last group, convert and store the tile.
+//   warps 1, 3  MMA issuers: 4 x tcgen05.mma (K = 32 each) per K group into one of two TMEM
+//               partial buffers (a fresh accumulation per group), then tcgen05.commit; warp 1
+//               issues the groups of buffer 0, warp 3 those of buffer 1.  An issuing warp slows
+//               the promotion warps of its SM sub-partition (which gate every buffer hand-back),
+//               so the issuing is split over two sub-partitions.
+//   warps 4..   promotion (2 or 4 warpgroups): tcgen05.ld the partial of group kb while the
+//               tensor cores fill the other buffer, fold in the scales and accumulate in
+//               registers (each warp owns 32 rows x BN/kPW columns); after the last group,
+//               convert and store the tile.
 // The CTA is persistent (one per SM) and walks a static tile list, so the epilogue of one
 // tile overlaps the first MMAs of the next.  setmaxnreg moves registers from the producer /
-// MMA warpgroup (40 each) to the two promotion warpgroups (232 each).
+// MMA warpgroup to the promotion warpgroups (see GemmShape).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -103,9 +107,16 @@ struct GemmShape {
     static constexpr int kStageBytes = kABytes + kBBytes;
     static constexpr int kStages = (BN == 256) ? 4 : 6;
     static constexpr int kScaleStages = (MODE == kModeWgrad) ? 4 : 0;
-    static constexpr int kHalf = BN / 2;           // columns per promotion warp
+    // Promotion warpgroups.  Each owns BN / kPW columns of the tile (all 128 rows; warp w of a
+    // group reads TMEM lanes 32*(w%4) ..).  Two: four groups (640 threads) halve each thread's
+    // arithmetic per K group but not its TMEM round trips, which set the fold's length; with
+    // 104 registers per thread they measured 6-8 % slower on the linear-layer shapes.
+    static constexpr int kPW = 2;
+    static constexpr int kPromoWarps = 4 * kPW;
+    static constexpr int kPromoThreads = 128 * kPW;
+    static constexpr int kCols = BN / kPW;         // columns per promotion thread
     static constexpr int kTmemCols = 2 * BN;       // two partial buffers
-    static constexpr int kThreads = 384;
+    static constexpr int kThreads = 128 + kPromoThreads;
     static constexpr int kMaxGroups = 1024;
     static constexpr int kOffScales = kStages * kStageBytes;
     static constexpr int kOffBars = kOffScales + kScaleStages * BN * 4;
@@ -115,14 +126,17 @@ struct GemmShape {
     // Epilogue staging: 2 KB per promotion warp and buffer, 1024-byte aligned (the 64-byte
     // swizzle of the tensor store works on absolute shared-memory address bits).  Two buffers per
     // warp where shared memory allows, so one slab's store reads while the next is written.
-    static constexpr int kEpiBufs = (MODE == kModeWgrad || GROUPED) ? 1 : 2;
+    static constexpr int kEpiBufs = (MODE == kModeWgrad || GROUPED || kPW == 4) ? 1 : 2;
     static constexpr int kOffEpi = (kOffGroups + (GROUPED ? 2 * (kMaxGroups + 1) * 4 : 0) + 1023) / 1024 * 1024;
-    static constexpr int kSmemBytes = kOffEpi + 8 * 2048 * kEpiBufs + 1024;
-    // Registers: launched at 168 per thread (384 x 168 = 64512); 128 x 40 + 256 x 232 = 64512.
-    static constexpr int kRegsLow = 40;
-    static constexpr int kRegsHigh = 232;
-    static constexpr int kRegsLaunch = 168;
-    static_assert(kThreads * kRegsLaunch >= 128 * kRegsLow + 256 * kRegsHigh, "register split");
+    static constexpr int kSmemBytes = kOffEpi + kPromoWarps * 2048 * kEpiBufs + 1024;
+    // Registers (setmaxnreg moves them from the producer / MMA warpgroup to the promotion
+    // warpgroups within the launch allocation):
+    //   384 threads launched at 168:  128 x 40 + 256 x 232 = 64512 <= 384 x 168
+    //   640 threads launched at  96:  128 x 56 + 512 x 104 = 60416 <= 640 x  96
+    static constexpr int kRegsLow = (kPW == 4) ? 56 : 40;
+    static constexpr int kRegsHigh = (kPW == 4) ? 104 : 232;
+    static constexpr int kRegsLaunch = (kPW == 4) ? 96 : 168;
+    static_assert(kThreads * kRegsLaunch >= 128 * kRegsLow + kPromoThreads * kRegsHigh, "register split");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
@@ -165,7 +179,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 }
 
 template <int MODE, int BN, bool GROUPED>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(GemmShape<MODE, BN, GROUPED>::kThreads, 1)
 gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmD, const GemmArgs args)
 {
@@ -200,14 +214,14 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull_bar(b), 1);
-            mbar_init(tempty_bar(b), 8);
+            mbar_init(tempty_bar(b), S::kPromoWarps);
         }
         for (int s = 0; s < S::kScaleStages; ++s) {
             mbar_init(sfull_bar(s), 1);
-            mbar_init(sempty_bar(s), 8);
+            mbar_init(sempty_bar(s), S::kPromoWarps);
         }
-        mbar_init(drain_bar, 1);
-        mbar_init(parked_bar, 8);
+        mbar_init(drain_bar, 2);
+        mbar_init(parked_bar, S::kPromoWarps);
         misc[1] = 0;
         misc[2] = 0;
         fence_mbar_init();
@@ -309,8 +323,11 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                 while (globaltimer_ns() - t0 < 50000ull) __nanosleep(1000);
             }
         }
-        } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
+        } else if (warp == 1 || warp == 3) {
+        // ------------------------------------------------------------ MMA issuers
+        // Warp 1 issues the K groups that accumulate into TMEM buffer 0, warp 3 those into buffer
+        // 1 (independent accumulators), so the issuing work is split over two SM sub-partitions.
+        const int mybuf = (warp == 1) ? 0 : 1;
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_e4m3_f32(BN, MODE == kModeDgrad);
             int stage = 0, tb = 0;
@@ -320,43 +337,49 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
             WorkItem it;
             while (ok && sched_next(ws, num_tiles, KB, it)) {
                 for (int kb = it.kb0; kb < it.kb1; ++kb) {
-                    if (!mbar_wait(tempty_bar(tb), tph ^ 1u, abort_flag)) { ok = false; break; }
-                    if (!mbar_wait(full_bar(stage), phase, abort_flag)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t sa = smem_u32(smem + stage * S::kStageBytes);
-                    const uint32_t sb = sa + S::kABytes;
-                    const uint32_t d = tmem_base + (uint32_t)(tb * BN);
+                    if (tb == mybuf) {
+                        if (!mbar_wait(tempty_bar(tb), tph ^ 1u, abort_flag)) { ok = false; break; }
+                        if (!mbar_wait(full_bar(stage), phase, abort_flag)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint32_t sa = smem_u32(smem + stage * S::kStageBytes);
+                        const uint32_t sb = sa + S::kABytes;
+                        const uint32_t d = tmem_base + (uint32_t)(tb * BN);
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const uint64_t ad = sdesc_sw128(sa + k * 32, 16, 1024);
-                        const uint64_t bd = (MODE == kModeDgrad) ? sdesc_sw128(sb + k * 4096, 16384, 1024)
-                                                                 : sdesc_sw128(sb + k * 32, 16, 1024);
-                        mma_f8f6f4(d, ad, bd, idesc, k > 0 ? 1u : 0u);
+                        for (int k = 0; k < 4; ++k) {
+                            const uint64_t ad = sdesc_sw128(sa + k * 32, 16, 1024);
+                            const uint64_t bd = (MODE == kModeDgrad) ? sdesc_sw128(sb + k * 4096, 16384, 1024)
+                                                                     : sdesc_sw128(sb + k * 32, 16, 1024);
+                            mma_f8f6f4(d, ad, bd, idesc, k > 0 ? 1u : 0u);
+                        }
+                        tc_commit(empty_bar(stage));
+                        tc_commit(tfull_bar(tb));
                     }
-                    tc_commit(empty_bar(stage));
-                    tc_commit(tfull_bar(tb));
                     if (++stage == S::kStages) { stage = 0; phase ^= 1u; }
                     if (++tb == 2) { tb = 0; tph ^= 1u; }
                 }
             }
-            // Drain: every MMA this thread issued has completed before TMEM is released.
+            // Drain: every MMA both issuers started has completed before TMEM is released.
             tc_commit(drain_bar);
-            const uint64_t t0 = globaltimer_ns();
-            while (!mbar_try_wait(drain_bar, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+            if (warp == 1) {
+                const uint64_t t0 = globaltimer_ns();
+                while (!mbar_try_wait(drain_bar, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+                }
             }
         }
         __syncwarp();
-        // Release TMEM once the promotion warps have read their last partial.
-        named_bar_sync(1, 32 + 256);
-        tc_fence_after();
-        tmem_dealloc(tmem_base, S::kTmemCols);
+        if (warp == 1) {
+            // Release TMEM once the promotion warps have read their last partial.
+            named_bar_sync(1, 32 + S::kPromoThreads);
+            tc_fence_after();
+            tmem_dealloc(tmem_base, S::kTmemCols);
+        }
         }
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(S::kRegsHigh));
         // ------------------------------------------------------------ promotion + epilogue
         const int pw = warp - 4;
         const int quad = warp & 3;            // TMEM lanes 32*quad .. 32*quad+31
-        const int half = pw >> 2;             // columns [half*BN/2, (half+1)*BN/2)
+        const int half = pw >> 2;             // column group: [half*kCols, (half+1)*kCols)
         const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
         const int rit = quad * 32 + lane;     // row within the tile
         const int ptid = pw * 32 + lane;      // promotion thread 0..255
@@ -364,19 +387,19 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
         uint32_t tph = 0, sph = 0;
         // Columns per TMEM load.  Each load is a round trip on the promotion's critical path,
         // so chunks are as wide as the registers allow: two 32-column chunks in flight beside
-        // the BN/2 accumulators.
+        // the accumulators (16 with four promotion warpgroups, whose threads have fewer registers).
         //
         // Wgrad multiplies every element by its own column's scale, which comes from shared
-        // memory; with one row per thread each thread would need all BN/2 column scales per K
+        // memory; with one row per thread each thread would need all its kCols column scales per K
         // group.  So Wgrad reads TMEM with the 16x256b shape instead: a thread holds 4 rows
         // (t/4 + 8i of the warp's 32) x 2 columns of every 8-column block, i.e. needs a quarter
         // of the column scales (an 8-byte load per block).  Its chunk is 16 columns (16
         // registers); acc[kBlocks * i + j] is row i's column pair of block j.
-        constexpr int kCW = (MODE == kModeWgrad || S::kHalf < 32) ? 16 : 32;
-        constexpr int kChunks = S::kHalf / kCW;
-        constexpr int kBlocks = S::kHalf / 8;
+        constexpr int kCW = (MODE == kModeWgrad || S::kCols < 32 || S::kPW == 4) ? 16 : 32;
+        constexpr int kChunks = S::kCols / kCW;
+        constexpr int kBlocks = S::kCols / 8;
         const int wt0 = lane & 3, wt1 = lane >> 2;   // Wgrad: column pair and first row of a thread
-        float2 acc[S::kHalf / 2];
+        float2 acc[S::kCols / 2];
         WorkSched wsched = sched_begin(args);
         WorkItem it;
         bool alive = true;
@@ -384,7 +407,7 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
             const TileInfo ti = decode_tile<GROUPED>(it.tile, nb_tiles, BN, args, g_off, g_pre);
             const int row = ti.row0 + rit;
             const bool in_a = row < args.M;
-            const int ncol0 = ti.n0 + half * S::kHalf;
+            const int ncol0 = ti.n0 + half * S::kCols;
             const float* sa_ptr = args.sA + (in_a ? row : 0);
             const float* sb_ptr = args.sB;
             size_t sb_step = 0;
@@ -396,7 +419,7 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                 sb_step = (size_t)(args.N >> 7);
             }
 #pragma unroll
-            for (int i = 0; i < S::kHalf / 2; ++i) acc[i] = make_float2(0.0f, 0.0f);
+            for (int i = 0; i < S::kCols / 2; ++i) acc[i] = make_float2(0.0f, 0.0f);
             // The row and block scales of the item's groups are pulled into L2 up front (one line
             // per group holds this warp's 32 row scales), so the per-group loads below, issued one
             // group ahead, find them there instead of in HBM.
@@ -418,8 +441,8 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                     if (!warp_wait(sfull_bar(ss), sph, abort_flag)) { ok = false; break; }
                 }
                 tc_fence_after();
-                const uint32_t taddr = tmem_base + lane_base + (uint32_t)(tb * BN + half * S::kHalf);
-                const float* cs = col_scales + ss * BN + half * S::kHalf;
+                const uint32_t taddr = tmem_base + lane_base + (uint32_t)(tb * BN + half * S::kCols);
+                const float* cs = col_scales + ss * BN + half * S::kCols;
                 const float2 c2 = make_float2(sa * sbv, sa * sbv);
                 // Wgrad: the row scales of this thread's 4 rows, from the lanes that loaded them.
                 float2 sa2w[4];
@@ -504,8 +527,8 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                 // interleaved by promotion thread: each warp store moves 512 contiguous bytes.
                 float4* slot = reinterpret_cast<float4*>(args.ws + (size_t)blockIdx.x * (128 * BN)) + ptid;
 #pragma unroll
-                for (int j = 0; j < S::kHalf / 2; j += 2)
-                    __stcg(slot + (j / 2) * 256, make_float4(acc[j].x, acc[j].y, acc[j + 1].x, acc[j + 1].y));
+                for (int j = 0; j < S::kCols / 2; j += 2)
+                    __stcg(slot + (j / 2) * S::kPromoThreads, make_float4(acc[j].x, acc[j].y, acc[j + 1].x, acc[j + 1].y));
                 __threadfence();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(parked_bar);
@@ -530,8 +553,8 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                     __syncwarp();   // orders the lanes' loads of the slot after lane 0's acquire
                     const float4* slot = reinterpret_cast<const float4*>(args.ws + (size_t)j * (128 * BN)) + ptid;
 #pragma unroll
-                    for (int q = 0; q < S::kHalf / 2; q += 2) {
-                        const float4 v = __ldcg(slot + (q / 2) * 256);
+                    for (int q = 0; q < S::kCols / 2; q += 2) {
+                        const float4 v = __ldcg(slot + (q / 2) * S::kPromoThreads);
                         acc[q].x += v.x;
                         acc[q].y += v.y;
                         acc[q + 1].x += v.z;
@@ -540,7 +563,7 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                 }
                 if (!alive) break;
             }
-            // Epilogue.  The warp's 32 rows x BN/2 columns leave through 2 KB staging buffers in
+            // Epilogue.  The warp's 32 rows x kCols columns leave through 2 KB staging buffers in
             // shared memory, one 32-row x 64-byte slab at a time.  16-byte unit p of staged row r
             // sits at unit 4r + (p ^ ((r >> 1) & 3)) -- the tensor map's 64-byte swizzle, and
             // conflict-free for the row-per-lane writes.  Dense GEMMs hand each slab to a bulk
@@ -553,7 +576,7 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                 uint4* stage0 = reinterpret_cast<uint4*>(smem + S::kOffEpi) + pw * 128 * S::kEpiBufs;
                 const int wrow0 = ti.row0 + quad * 32;
 #pragma unroll
-                for (int sl = 0; sl < S::kHalf / kSlabCols; ++sl) {
+                for (int sl = 0; sl < S::kCols / kSlabCols; ++sl) {
                     uint4* stage = stage0 + (sl % S::kEpiBufs) * 128;
                     uint4 u[4];
 #pragma unroll
@@ -621,7 +644,7 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
         if (!GROUPED && lane == 0) bulk_wait_group<0>();
         __syncwarp();
         tc_fence_before();
-        named_bar_arrive(1, 32 + 256);
+        named_bar_arrive(1, 32 + S::kPromoThreads);
     }
 
 }
