@@ -3,10 +3,11 @@
 
 Workload (one "step"): the DeepSeek-V3 expert-FFN up-projection linear layer with 4096 tokens,
 C_in = 7168, C_out = 2048, bf16 operands resident in HBM:
-    act 1x128 + 128x1^T (X, one pass) -> weight 128x128 (W) -> Fprop Y = X W^T (bf16 [4096, 2048])
-    act 1x128 + 128x1^T (dY, one pass)                     -> Dgrad dX = dY W  (bf16 [4096, 7168])
-                                                              Wgrad dW = dY^T X (fp32 [2048, 7168])
-6 kernel launches (8 with --separate-quant, which quantises each form in its own launch).  value = GEMM FLOPs (3 x 2*4096*2048*7168) / device time of the step.
+    X to 1x128 + 128x1^T and W to 128x128, one launch -> Fprop Y = X W^T (bf16 [4096, 2048])
+    dY to 1x128 + 128x1^T, one launch                 -> Dgrad dX = dY W  (bf16 [4096, 7168])
+                                                         Wgrad dW = dY^T X (fp32 [2048, 7168])
+5 kernel launches (8 with --separate-quant, which quantises each form of each tensor in its own
+launch).  value = GEMM FLOPs (3 x 2*4096*2048*7168) / device time of the step.
 L2 is flushed between steps, outside the timed step: a 256 MiB write, then a 256 MiB read of another
 buffer, so each step starts with a cold L2 that holds no dirty lines of the flush itself.
 
@@ -145,8 +146,7 @@ class ClockSampler:
 # ------------------------------------------------------------------------------------------ #
 # GPU arm
 # ------------------------------------------------------------------------------------------ #
-OPS_FUSED = ["act_dual_X", "weight_128x128_W", "gemm_fprop", "act_dual_dY", "gemm_dgrad",
-             "gemm_wgrad"]
+OPS_FUSED = ["quant_forward_XW", "gemm_fprop", "act_dual_dY", "gemm_dgrad", "gemm_wgrad"]
 OPS_SEPARATE = ["act_1x128_X", "weight_128x128_W", "gemm_fprop", "act_1x128_dY", "gemm_dgrad",
                 "act_128x1t_X", "act_128x1t_dY", "gemm_wgrad"]
 
@@ -182,6 +182,8 @@ def step_ops(ops, t, b, separate=False):
         "gemm_wgrad": lambda: ops.gemm_blockscaled(ops.WGRAD, b["dYtq"], b["sdYt"], b["Xtq"], b["sXt"], b["dW"]),
     }
     quant = {
+        "quant_forward_XW": lambda: ops.quant_forward(t["X"], t["W"], b["Xq"], b["sX"], b["Xtq"], b["sXt"],
+                                                      b["Wq"], b["sW"]),
         "act_dual_X": lambda: ops.act_dual(t["X"], b["Xq"], b["sX"], b["Xtq"], b["sXt"]),
         "act_dual_dY": lambda: ops.act_dual(t["dY"], b["dYq"], b["sdY"], b["dYtq"], b["sdYt"]),
         "act_1x128_X": lambda: ops.act_1x128(t["X"], b["Xq"], b["sX"]),
@@ -198,6 +200,7 @@ def step_ops(ops, t, b, separate=False):
 def op_work():
     """Algorithmic work per launch: ('flop', F) or ('bytes', B)."""
     return {
+        "quant_forward_XW": ("bytes", T_TOK * C_IN * QB_DUAL + C_OUT * C_IN * QB_128x128),
         "act_dual_X": ("bytes", T_TOK * C_IN * QB_DUAL),
         "act_dual_dY": ("bytes", T_TOK * C_OUT * QB_DUAL),
         "act_1x128_X": ("bytes", T_TOK * C_IN * QB_1x128),

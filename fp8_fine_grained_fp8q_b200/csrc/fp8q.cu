@@ -396,6 +396,23 @@ int fp8q_act_dual(const uint16_t* x, int64_t T, int64_t C, uint8_t* q, float* s,
     return launch_kernel(act_dual_kernel, grid, dim3(256), 0, (cudaStream_t)stream, false, x, q, s, qt, st, T, C);
 }
 
+int fp8q_quant_forward(const uint16_t* x, int64_t T, int64_t C, uint8_t* xq, float* xs, uint8_t* xqt, float* xst,
+                       const uint16_t* w, int64_t N, uint8_t* wq, float* ws, uint8_t* wqt_or_null,
+                       fp8q_stream_t stream)
+{
+    if (T < 0 || C < 0 || N < 0) return FP8Q_ERR_ARG;
+    if (T % 128 != 0 || C % 128 != 0 || N % 128 != 0) return FP8Q_ERR_SHAPE;
+    if (C == 0 || (T == 0 && N == 0)) return FP8Q_OK;
+    if (!x || !xq || !xs || !xqt || !xst || !w || !wq || !ws) return FP8Q_ERR_ARG;
+    if (!aligned16(x) || !aligned16(xq) || !aligned16(xs) || !aligned16(xqt) || !aligned16(xst) || !aligned16(w) ||
+        !aligned16(wq) || !aligned16(ws) || !aligned16(wqt_or_null))
+        return FP8Q_ERR_ALIGN;
+    const int64_t tiles = (T / 128 + N / 128) * (C / 128);
+    if (tiles > 0x7FFFFFFF) return FP8Q_ERR_UNSUPPORTED;
+    return launch_kernel(forward_operands_kernel, dim3((unsigned)tiles), dim3(256), 0, (cudaStream_t)stream, false, x,
+                         xq, xs, xqt, xst, T, C, w, wq, ws, wqt_or_null, N);
+}
+
 int fp8q_weight_128x128(const uint16_t* w, int64_t N, int64_t K, uint8_t* q, float* s, uint8_t* qt_or_null,
                         fp8q_stream_t stream)
 {

@@ -195,17 +195,13 @@ __global__ void __launch_bounds__(256) act_128x1_t_kernel(const uint16_t* __rest
 // lane, then one all-reduce step) leaves the maximum of row 16w + (l >> 1) on lanes 2r, 2r+1.
 // Codes: rows as 4-byte stores (128 B per warp row), columns as 16-byte stores of 16 tokens.
 // ------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(256, 3) act_dual_kernel(const uint16_t* __restrict__ x,
-                                                       uint8_t* __restrict__ q, float* __restrict__ s,
-                                                       uint8_t* __restrict__ qt, float* __restrict__ st,
-                                                       int64_t T, int64_t C)
+// One 128x128 tile (column block cb, token block tb) of the dual quantiser; red [8][128] and
+// inv_c [128] are this CTA's shared scratch.
+__device__ __forceinline__ void act_dual_tile(const uint16_t* __restrict__ x, uint8_t* __restrict__ q,
+                                              float* __restrict__ s, uint8_t* __restrict__ qt,
+                                              float* __restrict__ st, int64_t T, int64_t C, int64_t cb,
+                                              int64_t tb, float (*red)[128], float* inv_c)
 {
-    griddep_launch_dependents();
-    griddep_wait();
-    __shared__ __align__(16) float red[8][128];
-    __shared__ __align__(16) float inv_c[128];
-
-    const int64_t cb = blockIdx.x, tb = blockIdx.y;
     const int64_t c0 = cb * 128, t0 = tb * 128;
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t trow = t0 + 16 * w;
@@ -300,21 +296,29 @@ __global__ void __launch_bounds__(256, 3) act_dual_kernel(const uint16_t* __rest
         *reinterpret_cast<uint4*>(dst + (size_t)j * (size_t)T) = make_uint4(c[j][0], c[j][1], c[j][2], c[j][3]);
 }
 
+__global__ void __launch_bounds__(256, 3) act_dual_kernel(const uint16_t* __restrict__ x,
+                                                       uint8_t* __restrict__ q, float* __restrict__ s,
+                                                       uint8_t* __restrict__ qt, float* __restrict__ st,
+                                                       int64_t T, int64_t C)
+{
+    griddep_launch_dependents();
+    griddep_wait();
+    __shared__ __align__(16) float red[8][128];
+    __shared__ __align__(16) float inv_c[128];
+    act_dual_tile(x, q, s, qt, st, T, C, blockIdx.x, blockIdx.y, red, inv_c);
+}
+
 // ------------------------------------------------------------------------------------------
 // 128x128: w[N,K] -> q[N,K], s[N/128][K/128] (+ optional qt[K,N]).  One CTA per block; each
 // thread holds 64 of the block's 16384 values in registers, so the block is read once.
 // ------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) weight_128x128_kernel(const uint16_t* __restrict__ w,
-                                                             uint8_t* __restrict__ q,
-                                                             float* __restrict__ s,
-                                                             uint8_t* __restrict__ qt, int64_t N, int64_t K)
+// One 128x128 block (column block kb, row block nb) of the weight quantiser; red [8] and
+// codes [128][144] are this CTA's shared scratch (codes only when qt is requested).
+__device__ __forceinline__ void weight_tile(const uint16_t* __restrict__ w, uint8_t* __restrict__ q,
+                                            float* __restrict__ s, uint8_t* __restrict__ qt, int64_t N,
+                                            int64_t K, int64_t kb, int64_t nb, float* red,
+                                            uint8_t (*codes)[128 + 16])
 {
-    griddep_launch_dependents();
-    griddep_wait();
-    __shared__ float red[8];
-    __shared__ __align__(16) uint8_t codes[128][128 + 16];
-
-    const int64_t kb = blockIdx.x, nb = blockIdx.y;
     const int64_t KB = K >> 7;
     const int tid = threadIdx.x;
     const uint16_t* wb = w + nb * 128 * K + kb * 128;
@@ -365,6 +369,47 @@ __global__ void __launch_bounds__(256) weight_128x128_kernel(const uint16_t* __r
             }
             reinterpret_cast<uint4*>(dst)[p] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
         }
+    }
+}
+
+__global__ void __launch_bounds__(256) weight_128x128_kernel(const uint16_t* __restrict__ w,
+                                                             uint8_t* __restrict__ q,
+                                                             float* __restrict__ s,
+                                                             uint8_t* __restrict__ qt, int64_t N, int64_t K)
+{
+    griddep_launch_dependents();
+    griddep_wait();
+    __shared__ float red[8];
+    __shared__ __align__(16) uint8_t codes[128][128 + 16];
+    weight_tile(w, q, s, qt, N, K, blockIdx.x, blockIdx.y, red, codes);
+}
+
+// ------------------------------------------------------------------------------------------
+// The forward operands of a linear layer Y = X W^T in one launch: x[T,C] to both activation
+// forms (as act_dual_kernel) and w[N,C] to 128x128 blocks (as weight_128x128_kernel).  CTA b
+// takes dual tile b (token-block-major) while b < tiles_x, then weight block b - tiles_x; one
+// grid instead of two saves a launch and a partly filled last wave.
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256, 3) forward_operands_kernel(
+    const uint16_t* __restrict__ x, uint8_t* __restrict__ xq, float* __restrict__ xs, uint8_t* __restrict__ xqt,
+    float* __restrict__ xst, int64_t T, int64_t C, const uint16_t* __restrict__ w, uint8_t* __restrict__ wq,
+    float* __restrict__ ws, uint8_t* __restrict__ wqt, int64_t N)
+{
+    griddep_launch_dependents();
+    griddep_wait();
+    __shared__ __align__(16) uint8_t scratch[128 * (128 + 16) + 8 * 4];
+    const int64_t CB = C >> 7;
+    const int64_t tiles_x = CB * (T >> 7);
+    const int64_t b = blockIdx.x;
+    if (b < tiles_x) {
+        float (*red)[128] = reinterpret_cast<float (*)[128]>(scratch);
+        float* inv_c = reinterpret_cast<float*>(scratch + 8 * 128 * 4);
+        act_dual_tile(x, xq, xs, xqt, xst, T, C, b % CB, b / CB, red, inv_c);
+    } else {
+        const int64_t bw = b - tiles_x;
+        uint8_t (*codes)[128 + 16] = reinterpret_cast<uint8_t (*)[128 + 16]>(scratch);
+        float* red = reinterpret_cast<float*>(scratch + 128 * (128 + 16));
+        weight_tile(w, wq, ws, wqt, N, C, bw % CB, bw / CB, red, codes);
     }
 }
 

@@ -47,6 +47,7 @@ def lib() -> ctypes.CDLL:
         "fp8q_act_1x128": [P, I64, I64, P, P, P],
         "fp8q_act_128x1_transposed": [P, I64, I64, P, P, P],
         "fp8q_act_dual": [P, I64, I64, P, P, P, P, P],
+        "fp8q_quant_forward": [P, I64, I64, P, P, P, P, P, I64, P, P, P, P],
         "fp8q_weight_128x128": [P, I64, I64, P, P, P, P],
         "fp8_gemm_blockscaled": [I, P, P, P, P, P, I64, I64, I64, P, ctypes.c_size_t, P],
         "fp8_grouped_gemm_blockscaled": [P, P, P, P, P, I32, I64, I64, I64, P, P],
@@ -141,6 +142,31 @@ def act_dual(x: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tensor | N
     _check("fp8q_act_dual",
            lib().fp8q_act_dual(_p(x), T, C, _p(q), _p(s), _p(qt), _p(st), _stream(x.device)))
     return q, s, qt, st
+
+
+def quant_forward(x: torch.Tensor, w: torch.Tensor, xq=None, xs=None, xqt=None, xst=None,
+                  wq=None, ws=None, wqt=None, transposed_w: bool = False):
+    """x[T,C], w[N,C] bf16 -> ((xq, xs, xqt, xst), (wq, ws, wqt or None)) in one launch: the outputs of
+    act_dual(x) and weight_128x128(w), bit for bit."""
+    _require(x, "x", torch.bfloat16, 2)
+    _require(w, "w", torch.bfloat16, 2)
+    T, C = x.shape
+    N, Cw = w.shape
+    if Cw != C:
+        raise ValueError("x and w must share the inner dimension")
+    dev = x.device
+    xq = _out(xq, (T, C), torch.uint8, dev, "xq")
+    xs = _out(xs, (C // 128, T), torch.float32, dev, "xs")
+    xqt = _out(xqt, (C, T), torch.uint8, dev, "xqt")
+    xst = _out(xst, (T // 128, C), torch.float32, dev, "xst")
+    wq = _out(wq, (N, C), torch.uint8, dev, "wq")
+    ws = _out(ws, (N // 128, C // 128), torch.float32, dev, "ws")
+    if transposed_w or wqt is not None:
+        wqt = _out(wqt, (C, N), torch.uint8, dev, "wqt")
+    _check("fp8q_quant_forward",
+           lib().fp8q_quant_forward(_p(x), T, C, _p(xq), _p(xs), _p(xqt), _p(xst), _p(w), N, _p(wq), _p(ws),
+                                    _p(wqt), _stream(dev)))
+    return (xq, xs, xqt, xst), (wq, ws, wqt)
 
 
 def weight_128x128(w: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tensor | None = None,

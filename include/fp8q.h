@@ -122,6 +122,20 @@ FP8Q_API int fp8q_act_dual(const uint16_t* x, int64_t T, int64_t C, uint8_t* q, 
                            uint8_t* qt, float* st, fp8q_stream_t stream);
 
 /*
+ * The forward operands of a linear layer Y = X W^T in one launch: X to both activation forms
+ * (exactly as fp8q_act_dual) and W to 128x128 blocks (exactly as fp8q_weight_128x128 with
+ * K = C).  Outputs are bit-identical to the two separate calls; one launch instead of two
+ * saves a launch and a partly filled last wave.
+ *   x : [T, C] bf16   -> xq [T, C], xs [C/128, T], xqt [C, T], xst [T/128, C]
+ *   w : [N, C] bf16   -> wq [N, C], ws [N/128, C/128], wqt [C, N] (optional: NULL skips it)
+ * T, C, N multiples of 128 (FP8Q_ERR_SHAPE otherwise).  All pointers 16-byte aligned, caller-owned,
+ * device.
+ */
+FP8Q_API int fp8q_quant_forward(const uint16_t* x, int64_t T, int64_t C, uint8_t* xq, float* xs, uint8_t* xqt,
+                                float* xst, const uint16_t* w, int64_t N, uint8_t* wq, float* ws,
+                                uint8_t* wqt_or_null, fp8q_stream_t stream);
+
+/*
  * 128x128 block-wise weight quantisation ([SUMMARY] Key ideas, FP8 bullet).
  *   w : [N, K] bf16            q : [N, K] E4M3 codes         s : [N/128, K/128] fp32 scales
  *   qt_or_null : NULL, or [K, N] receiving the same codes transposed.

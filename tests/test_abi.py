@@ -82,6 +82,18 @@ def test_act_dual_host_checks(L):
     assert d(P(FAKE), 128 * 65536, 128, P(FAKE), P(FAKE), P(FAKE), P(FAKE), s) == ERR_UNSUPPORTED
 
 
+def test_quant_forward_host_checks(L):
+    f = L.fp8q_quant_forward
+    a = [P(FAKE)] * 5
+    b = [P(FAKE)] * 3
+    assert f(P(FAKE), 128, 100, *a[1:], P(FAKE), 128, *b, None, None) == ERR_SHAPE
+    assert f(P(FAKE), 128, 128, *a[1:], P(FAKE), 100, *b, None, None) == ERR_SHAPE
+    assert f(P(FAKE), -128, 128, *a[1:], P(FAKE), 128, *b, None, None) == ERR_ARG
+    assert f(P(FAKE), 128, 128, *a[1:], None, 128, *b, None, None) == ERR_ARG
+    assert f(P(FAKE), 128, 128, *a[1:], P(FAKE), 128, P(FAKE), P(FAKE), P(MISALIGNED), None) == ERR_ALIGN
+    assert f(P(FAKE), 0, 128, *a[1:], P(FAKE), 0, *b, None, None) == OK
+
+
 def test_weight_host_checks(L):
     s = None
     assert L.fp8q_weight_128x128(P(FAKE), 100, 128, P(FAKE), P(FAKE), None, s) == ERR_SHAPE

@@ -161,6 +161,39 @@ def test_act_dual_full_size(which):
     check_dual(bits, f"{which}{bits.shape}")
 
 
+def check_forward(xbits, wbits, transposed, what):
+    x, w = bf16_dev(xbits), bf16_dev(wbits)
+    T, C = xbits.shape
+    N = wbits.shape[0]
+    (xq, xs, xqt, xst), (wq, ws, wqt) = ops.quant_forward(
+        x, w, _poison_q((T, C)), _poison_s((C // 128, T)), _poison_q((C, T)), _poison_s((T // 128, C)),
+        _poison_q((N, C)), _poison_s((N // 128, C // 128)), _poison_q((C, N)) if transposed else None)
+    torch.cuda.synchronize()
+    oq, os_ = oracle.quant_1x128(xbits)
+    oqt, ost = oracle.quant_128x1_t(xbits)
+    owq, ows, owqt = oracle.quant_128x128(wbits, want_transposed=transposed)
+    assert_same(host(xq), host(xs), oq, os_, f"forward x 1x128 {what}")
+    assert_same(host(xqt), host(xst), oqt, ost, f"forward x 128x1 {what}")
+    assert_same(host(wq), host(ws), owq, ows, f"forward w {what}")
+    if transposed:
+        assert np.array_equal(host(wqt), owqt), f"forward w transposed codes {what}"
+
+
+@pytest.mark.parametrize("T,C,N,transposed", [(128, 128, 128, True), (256, 384, 640, False), (384, 1024, 256, True)])
+def test_quant_forward_small(T, C, N, transposed):
+    check_forward(synth.activations_channel_outliers(T, C, seed=T + C + N),
+                  synth.weights(N, C, seed=T + 2 * N), transposed, f"{T}x{C}, N={N}")
+
+
+def test_quant_forward_special_values():
+    check_forward(special_values(256, 1024, seed=11), special_values(512, 1024, seed=13), True, "special")
+
+
+def test_quant_forward_full_size():
+    d = linear_layer_inputs()
+    check_forward(d["X"], d["W"], False, "linear layer")
+
+
 def run_weight(bits, transposed):
     w = bf16_dev(bits)
     N, K = bits.shape
