@@ -48,6 +48,16 @@ QB_128x128 = 2 + 1 + 4 / (128 * 128)
 QB_DUAL = 2 + 2 * (1 + 4 / 128)                  # one read, both code sets and scale sets
 
 
+def max_over_ranks(x: float, dist, device) -> float:
+    """The largest of every rank's x (all ranks call it, in the same order); x itself on one rank."""
+    if dist is None:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -286,10 +296,7 @@ def run_ours(args, rank, world, dist):
             per_op[name].append(bevs[s][i].elapsed_time(bevs[s][i + 1]))
     sum_step_ms = float(sum(step_ms))
     total_ms = start.elapsed_time(end)
-    if dist is not None:
-        tt = torch.tensor([sum_step_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        sum_step_ms = float(tt.item())
+    sum_step_ms = max_over_ranks(sum_step_ms, dist, dev)
     ms_per_step = sum_step_ms / args.steps
     value = world * STEP_FLOP / (ms_per_step * 1e-3) / 1e12
 
@@ -317,10 +324,7 @@ def run_ours(args, rank, world, dist):
         if s >= 2:
             e2e_ms.append(e0.elapsed_time(e1))
     e2e_sum = float(sum(e2e_ms))
-    if dist is not None:
-        tt = torch.tensor([e2e_sum], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_sum = float(tt.item())
+    e2e_sum = max_over_ranks(e2e_sum, dist, dev)
     e2e_value = world * STEP_FLOP / (e2e_sum / len(e2e_ms) * 1e-3) / 1e12
 
     peaks, peak_kind = load_peaks()
