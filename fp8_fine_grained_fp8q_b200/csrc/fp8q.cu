@@ -203,7 +203,7 @@ bool want_streamk(int64_t tiles, int ctas, int kb)
 template <int MODE, int BN, bool GROUPED>
 int launch_gemm(const uint8_t* A, const float* sA, const uint8_t* B, const float* sB, void* D,
                 const int32_t* offsets, int E, int64_t M, int64_t N, int64_t K, cudaStream_t st,
-                void* workspace = nullptr, size_t ws_bytes = 0)
+                void* workspace = nullptr, size_t ws_bytes = 0, bool accumulate = false)
 {
     using S = GemmShape<MODE, BN, GROUPED>;
     const int prep = prepare_kernel<MODE, BN, GROUPED>();
@@ -233,6 +233,7 @@ int launch_gemm(const uint8_t* A, const float* sA, const uint8_t* B, const float
     a.flags = nullptr;
     a.stamp = 0;
     a.units = 0;
+    a.accumulate = accumulate ? 1 : 0;
     const int sms = sm_count();
     if (sms <= 0) return FP8Q_ERR_CUDA;
     // Grouped: at most ceil(Mtot/128) + E row tiles (each group adds at most one partial tile).
@@ -272,11 +273,11 @@ int choose_bn(int64_t M, int64_t N, int extra_m_tiles)
 
 template <int MODE>
 int gemm_mode(const uint8_t* A, const float* sA, const uint8_t* B, const float* sB, void* D, int64_t M,
-              int64_t N, int64_t K, cudaStream_t st, void* ws, size_t ws_bytes)
+              int64_t N, int64_t K, cudaStream_t st, void* ws, size_t ws_bytes, bool accumulate = false)
 {
     if (choose_bn(M, N, 0) == 256)
-        return launch_gemm<MODE, 256, false>(A, sA, B, sB, D, nullptr, 1, M, N, K, st, ws, ws_bytes);
-    return launch_gemm<MODE, 128, false>(A, sA, B, sB, D, nullptr, 1, M, N, K, st, ws, ws_bytes);
+        return launch_gemm<MODE, 256, false>(A, sA, B, sB, D, nullptr, 1, M, N, K, st, ws, ws_bytes, accumulate);
+    return launch_gemm<MODE, 128, false>(A, sA, B, sB, D, nullptr, 1, M, N, K, st, ws, ws_bytes, accumulate);
 }
 
 // Waits on an mbarrier that nothing ever arrives on, so the bounded wait must expire, latch
@@ -439,7 +440,7 @@ size_t fp8q_gemm_workspace_size(int mode, int64_t M, int64_t N, int64_t K)
 int fp8_gemm_blockscaled(int mode, const uint8_t* A, const float* sA, const uint8_t* B, const float* sB, void* D,
                          int64_t M, int64_t N, int64_t K, void* workspace, size_t ws_bytes, fp8q_stream_t stream)
 {
-    if (mode != FP8Q_FPROP && mode != FP8Q_DGRAD && mode != FP8Q_WGRAD) return FP8Q_ERR_ARG;
+    if (mode != FP8Q_FPROP && mode != FP8Q_DGRAD && mode != FP8Q_WGRAD && mode != FP8Q_WGRAD_ACC) return FP8Q_ERR_ARG;
     if (M < 0 || N < 0 || K < 0) return FP8Q_ERR_ARG;
     if (N % 128 != 0 || K % 128 != 0) return FP8Q_ERR_SHAPE;
     if (M == 0 || N == 0) return FP8Q_OK;
@@ -447,7 +448,8 @@ int fp8_gemm_blockscaled(int mode, const uint8_t* A, const float* sA, const uint
     if (!A || !sA || !B || !sB || !D) return FP8Q_ERR_ARG;
     if (!aligned16(A) || !aligned16(sA) || !aligned16(B) || !aligned16(sB) || !aligned16(D)) return FP8Q_ERR_ALIGN;
     if (K == 0) {
-        // An empty contraction: D = 0.
+        // An empty contraction: D = 0 (D += 0 leaves it as it is).
+        if (mode == FP8Q_WGRAD_ACC) return FP8Q_OK;
         const size_t bytes = (size_t)M * (size_t)N * (mode == FP8Q_WGRAD ? 4u : 2u);
         return cudaMemsetAsync(D, 0, bytes, (cudaStream_t)stream) == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
     }
@@ -455,7 +457,8 @@ int fp8_gemm_blockscaled(int mode, const uint8_t* A, const float* sA, const uint
     switch (mode) {
     case FP8Q_FPROP: return gemm_mode<kModeFprop>(A, sA, B, sB, D, M, N, K, st, workspace, ws_bytes);
     case FP8Q_DGRAD: return gemm_mode<kModeDgrad>(A, sA, B, sB, D, M, N, K, st, workspace, ws_bytes);
-    default: return gemm_mode<kModeWgrad>(A, sA, B, sB, D, M, N, K, st, workspace, ws_bytes);
+    case FP8Q_WGRAD: return gemm_mode<kModeWgrad>(A, sA, B, sB, D, M, N, K, st, workspace, ws_bytes);
+    default: return gemm_mode<kModeWgrad>(A, sA, B, sB, D, M, N, K, st, workspace, ws_bytes, true);
     }
 }
 

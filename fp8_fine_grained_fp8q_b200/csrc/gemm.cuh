@@ -48,6 +48,7 @@ struct GemmArgs {
     unsigned long long* flags;   // per CTA: == stamp once its slot holds this launch's partial
     unsigned long long stamp; // unique per launch, so flags never need resetting
     int64_t units;            // tiles * KB
+    int32_t accumulate;       // Wgrad only: 1 adds the result into D (D += dY^T X), 0 overwrites D
 };
 
 // One piece of work: groups [kb0, kb1) of tile `tile`.
@@ -618,7 +619,10 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                         fence_proxy_async_smem();     // the writes above, before the async-proxy read
                         __syncwarp();
                         if (lane == 0) {
-                            tma_store_2d(&tmD, smem_u32(stage), ncol0 + sl * kSlabCols, wrow0);
+                            if (MODE == kModeWgrad && args.accumulate)
+                                tma_reduce_add_2d(&tmD, smem_u32(stage), ncol0 + sl * kSlabCols, wrow0);
+                            else
+                                tma_store_2d(&tmD, smem_u32(stage), ncol0 + sl * kSlabCols, wrow0);
                             bulk_commit_group();
                         }
                     } else {

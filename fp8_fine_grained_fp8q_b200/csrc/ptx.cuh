@@ -192,6 +192,15 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* tm, uint32_t src
                  : "memory");
 }
 
+// Like tma_store_2d, but each element of the box is added to the one in global memory (the
+// tensor map's element type, here FP32) instead of replacing it.
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* tm, uint32_t src, int32_t x, int32_t y)
+{
+    asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(tm),
+                 "r"(src), "r"(x), "r"(y)
+                 : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
 // Until at most N of this thread's bulk async-groups still read their shared-memory source.

@@ -17,7 +17,7 @@ import torch
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfp8q.so")
 
-FPROP, DGRAD, WGRAD = 0, 1, 2
+FPROP, DGRAD, WGRAD, WGRAD_ACC = 0, 1, 2, 3
 DEV_OK, DEV_TIMEOUT, DEV_BAD_OFFSETS = 0, 1, 2
 
 _lib = None
@@ -206,10 +206,13 @@ def gemm_workspace(mode: int, M: int, N: int, K: int, device: torch.device) -> t
 def gemm_blockscaled(mode: int, A: torch.Tensor, sA: torch.Tensor, B: torch.Tensor,
                      sB: torch.Tensor, out: torch.Tensor | None = None,
                      workspace: torch.Tensor | None = None):
-    """Block-scaled FP8 GEMM.  FPROP: B = W[N,K]; DGRAD: B = W[K,N]; WGRAD: B = X^T[N,K].
-    Returns D[M,N] (bf16, or fp32 for WGRAD).  `workspace` (uint8, CUDA) enables the stream-K
-    schedule; by default a per-device workspace sized by fp8q_gemm_workspace_size is used.
-    A workspace must not be shared by GEMMs that may run concurrently."""
+    """Block-scaled FP8 GEMM.  FPROP: B = W[N,K]; DGRAD: B = W[K,N]; WGRAD: B = X^T[N,K];
+    WGRAD_ACC: as WGRAD, added into `out` (required, fp32).
+    Returns D[M,N] (bf16, or fp32 for WGRAD / WGRAD_ACC).  `workspace` (uint8, CUDA) enables the
+    stream-K schedule; by default a per-device workspace sized by fp8q_gemm_workspace_size is
+    used.  A workspace must not be shared by GEMMs that may run concurrently."""
+    if mode == WGRAD_ACC and out is None:
+        raise ValueError("WGRAD_ACC accumulates into `out`: pass the fp32 gradient to add to")
     _require(A, "A", torch.uint8, 2)
     _require(B, "B", torch.uint8, 2)
     _require(sA, "sA", torch.float32, 2)
@@ -219,7 +222,7 @@ def gemm_blockscaled(mode: int, A: torch.Tensor, sA: torch.Tensor, B: torch.Tens
     Kb = B.shape[0] if mode == DGRAD else B.shape[1]
     if Kb != K:
         raise ValueError(f"inner dimensions differ: A has K={K}, B has {Kb}")
-    dtype = torch.float32 if mode == WGRAD else torch.bfloat16
+    dtype = torch.float32 if mode in (WGRAD, WGRAD_ACC) else torch.bfloat16
     out = _out(out, (M, N), dtype, A.device, "out")
     if workspace is None:
         workspace = gemm_workspace(mode, M, N, K, A.device)

@@ -74,11 +74,13 @@ enum {
     FP8Q_DEV_BAD_OFFSETS = 2   /* grouped GEMM: offsets not 0-based / nondecreasing / ending at Mtot */
 };
 
-/* GEMM modes (the three GEMMs of a linear layer, [REPOST] paragraph 2, Figure 6). */
+/* GEMM modes (the three GEMMs of a linear layer, [REPOST] paragraph 2, Figure 6; the FP32
+ * weight gradient is accumulated across micro-batches, [REPOST] paragraph 3). */
 enum {
     FP8Q_FPROP = 0,            /* Y  = X  W^T : D bf16 */
     FP8Q_DGRAD = 1,            /* dX = dY W   : D bf16 */
-    FP8Q_WGRAD = 2             /* dW = dY^T X : D fp32 */
+    FP8Q_WGRAD = 2,            /* dW = dY^T X : D fp32 */
+    FP8Q_WGRAD_ACC = 3         /* dW += dY^T X : D fp32, accumulated into (gradient accumulation) */
 };
 
 /* Human-readable name of a return code (static storage; never NULL). */
@@ -156,15 +158,22 @@ FP8Q_API int fp8q_weight_128x128(const uint16_t* w, int64_t N, int64_t K, uint8_
  *                    transposed, no requantisation; sB = [K/128, N/128]; D = bf16 [M, N].
  *   mode FP8Q_WGRAD: B = X^T [N, K] codes (128x1 along K = tokens), sB = [K/128, N];
  *                    D = fp32 [M, N].
+ *   mode FP8Q_WGRAD_ACC: as FP8Q_WGRAD, but the result is added into D (D must hold the
+ *                    FP32 gradient so far; each element gets one FP32 addition).
  * Requirements: K % 128 == 0, N % 128 == 0 (FP8Q_ERR_SHAPE); M >= 0 (any M, the last row tile
- * is masked); K/128 < 2^24.  D is fully overwritten (no accumulation into D).
- * workspace / ws_bytes: reserved for split-K schedules; pass NULL / 0.  fp8q_gemm_workspace_size
- * reports the bytes a call needs (currently always 0).
+ * is masked); M, N, K < 2^31 (FP8Q_ERR_UNSUPPORTED).  D is fully overwritten, except in
+ * FP8Q_WGRAD_ACC.  K == 0 writes D = 0 (FP8Q_WGRAD_ACC: leaves D unchanged).
+ * workspace / ws_bytes: optional scratch for the stream-K schedule (used when the output tiles do
+ * not fill whole waves of the persistent grid): at least fp8q_gemm_workspace_size(...) bytes,
+ * 256-byte aligned, device memory owned by the caller, reusable across calls on one stream
+ * (never cleared: each launch stamps its flags with a fresh value).  NULL / 0, or a smaller
+ * buffer, runs the data-parallel schedule instead -- same results, possibly slower.
  */
 FP8Q_API int fp8_gemm_blockscaled(int mode, const uint8_t* A, const float* sA, const uint8_t* B,
                          const float* sB, void* D, int64_t M, int64_t N, int64_t K,
                          void* workspace, size_t ws_bytes, fp8q_stream_t stream);
 
+/* Bytes of workspace fp8_gemm_blockscaled can use for a problem (0: none is useful). */
 FP8Q_API size_t fp8q_gemm_workspace_size(int mode, int64_t M, int64_t N, int64_t K);
 
 /*

@@ -107,6 +107,8 @@ def test_gemm_host_checks(L):
     g = L.fp8_gemm_blockscaled
     args = (P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE))
     assert g(7, *args, 128, 128, 128, None, 0, s) == ERR_ARG            # bad mode
+    assert g(4, *args, 128, 128, 128, None, 0, s) == ERR_ARG
+    assert g(3, *args, 128, 128, 0, None, 0, s) == OK                    # D += nothing: no launch
     assert g(0, *args, -1, 128, 128, None, 0, s) == ERR_ARG
     assert g(0, *args, 128, 100, 128, None, 0, s) == ERR_SHAPE
     assert g(1, *args, 128, 128, 96, None, 0, s) == ERR_SHAPE

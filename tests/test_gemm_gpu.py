@@ -18,7 +18,7 @@ from tests._util import check_gemm, f32_dev, host, linear_layer_inputs, u8_dev
 
 pytestmark = pytest.mark.gpu
 
-FPROP, DGRAD, WGRAD = ops.FPROP, ops.DGRAD, ops.WGRAD
+FPROP, DGRAD, WGRAD, WGRAD_ACC = ops.FPROP, ops.DGRAD, ops.WGRAD, ops.WGRAD_ACC
 
 
 # Kernel configurations: tile width x schedule (data-parallel whole tiles, or stream-K over
@@ -135,6 +135,59 @@ def test_exact_wgrad(T, Cout, Cin, bn, monkeypatch):
     assert np.array_equal(got, exact)
 
 
+def run_wgrad_acc(A, sA, B, sB, D0, times, bn=None, monkeypatch=None):
+    """D0 (fp32 [M, N]) plus `times` accumulating Wgrad calls."""
+    if bn is not None:
+        set_config(monkeypatch, bn)
+    D = torch.from_numpy(np.ascontiguousarray(D0, dtype=np.float32)).cuda()
+    for _ in range(times):
+        ops.gemm_blockscaled(WGRAD_ACC, u8_dev(A), f32_dev(sA), u8_dev(B), f32_dev(sB), out=D)
+    torch.cuda.synchronize()
+    assert ops.device_status() == ops.DEV_OK
+    return host(D).astype(np.float64)
+
+
+@pytest.mark.parametrize("bn", list(CONFIGS))
+def test_exact_wgrad_accumulate(bn, monkeypatch):
+    # Operands whose product P = dY^T X is exact in FP32 (as in test_exact_wgrad, where the plain
+    # mode must return P bit for bit).  Accumulating into D0 = P must give 2P, into D0 = -P zero:
+    # both sums are exact, so both are bit-exact checks of "D += P".
+    T, Cout, Cin = 512, 384, 512
+    g = np.random.Generator(np.random.PCG64(T + Cout * Cin))
+    dY = g.integers(-8, 9, size=(T, Cout)).astype(np.float32)
+    X = g.integers(-8, 9, size=(T, Cin)).astype(np.float32)
+    dY[1::128, :] = 0.0
+    X[0::128, :] = 0.0
+    dY[0::128, :] = 448.0
+    X[1::128, :] = -448.0
+    dY *= np.exp2(g.integers(-4, 5, size=Cout))[None, :].astype(np.float32)
+    X *= np.exp2(g.integers(-4, 5, size=Cin))[None, :].astype(np.float32)
+    P = dY.astype(np.float64).T @ X.astype(np.float64)
+    assert np.array_equal(P.astype(np.float32).astype(np.float64), P)
+    gq, gs = oracle.quant_128x1_t(_bits(dY))
+    xq, xs = oracle.quant_128x1_t(_bits(X))
+    assert np.array_equal(run_wgrad_acc(gq, gs, xq, xs, P, 1, bn, monkeypatch), 2.0 * P)
+    assert np.array_equal(run_wgrad_acc(gq, gs, xq, xs, -P, 1, bn, monkeypatch), np.zeros_like(P))
+
+
+@pytest.mark.parametrize("bn", list(CONFIGS))
+def test_wgrad_accumulate_within_tolerance(bn, monkeypatch):
+    T, Cout, Cin = 384, 384, 768
+    dY = synth.output_grad(T, Cout, seed=71)
+    X = synth.activations_channel_outliers(T, Cin, seed=72)
+    gq, gs = oracle.quant_128x1_t(dY)
+    xq, xs = oracle.quant_128x1_t(X)
+    ref, S = oracle.gemm(WGRAD, gq, gs, xq, xs)
+    D0 = np.random.Generator(np.random.PCG64(73)).standard_normal((Cout, Cin)).astype(np.float32) * 1e-3
+    got = run_wgrad_acc(gq, gs, xq, xs, D0, 1, bn, monkeypatch)
+    check_gemm(got, D0.astype(np.float64) + ref, S, f"wgrad accumulate {T}x{Cout}x{Cin}", bf16_out=False)
+
+
+def test_wgrad_accumulate_rejects_missing_out():
+    with pytest.raises(ValueError):
+        ops.gemm_blockscaled(WGRAD_ACC, *(torch.zeros(1, device="cuda"),) * 4)
+
+
 # ------------------------------------------------------------------------------------------ #
 # Tolerance cases, full outputs
 # ------------------------------------------------------------------------------------------ #
@@ -245,6 +298,9 @@ def test_full_wgrad():
     got = run_gemm(WGRAD, gq, gs, xq, xs)
     assert got.shape == (2048, 7168)
     sampled_check(WGRAD, gq, gs, xq, xs, got, "wgrad 2048x7168x4096")
+    # Accumulating into zeros adds each result to 0 exactly: bit-identical to the overwrite.
+    acc = run_wgrad_acc(gq, gs, xq, xs, np.zeros((2048, 7168), np.float32), 1)
+    assert np.array_equal(acc, got.astype(np.float64))
 
 
 @pytest.mark.parametrize("N", [1536, 512])
