@@ -129,7 +129,7 @@ bool make_tmap_u8(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t ou
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Row-major output matrix [outer][inner] of 2- or 4-byte elements, stored by the GEMM epilogue in
+// Row-major output matrix [outer][inner] of 1-, 2- or 4-byte elements, stored by the GEMM epilogue in
 // boxes of 32 rows x 64 bytes with the 64-byte swizzle.
 bool make_tmap_out(CUtensorMap* tm, void* base, uint64_t inner, uint64_t outer, int elt_bytes)
 {
@@ -139,7 +139,10 @@ bool make_tmap_out(CUtensorMap* tm, void* base, uint64_t inner, uint64_t outer, 
     const cuuint64_t strides[1] = {inner * (uint64_t)elt_bytes};
     const cuuint32_t box[2] = {(cuuint32_t)(64 / elt_bytes), 32};
     const cuuint32_t estr[2] = {1, 1};
-    return fn(tm, elt_bytes == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims,
+    const CUtensorMapDataType dt = elt_bytes == 4   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                   : elt_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                    : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    return fn(tm, dt, 2, base, dims,
               strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -203,7 +206,8 @@ bool want_streamk(int64_t tiles, int ctas, int kb)
 template <int MODE, int BN, bool GROUPED>
 int launch_gemm(const uint8_t* A, const float* sA, const uint8_t* B, const float* sB, void* D,
                 const int32_t* offsets, int E, int64_t M, int64_t N, int64_t K, cudaStream_t st,
-                void* workspace = nullptr, size_t ws_bytes = 0, bool accumulate = false)
+                void* workspace = nullptr, size_t ws_bytes = 0, bool accumulate = false,
+                uint8_t* q_out = nullptr, float* s_out = nullptr)
 {
     using S = GemmShape<MODE, BN, GROUPED>;
     const int prep = prepare_kernel<MODE, BN, GROUPED>();
@@ -216,10 +220,12 @@ int launch_gemm(const uint8_t* A, const float* sA, const uint8_t* B, const float
         const uint64_t rows = GROUPED ? (uint64_t)E * (uint64_t)N : (uint64_t)N;
         if (!make_tmap_u8(&tb, B, (uint64_t)K, rows, 128, BN)) return FP8Q_ERR_CUDA;
     }
-    CUtensorMap td;   // the epilogue's store map (the grouped GEMM stores without it)
+    CUtensorMap td, tq;   // the epilogue's store maps (the grouped GEMM stores without them)
     memset(&td, 0, sizeof(td));
-    if (!GROUPED && !make_tmap_out(&td, D, (uint64_t)N, (uint64_t)M, MODE == kModeWgrad ? 4 : 2))
+    memset(&tq, 0, sizeof(tq));
+    if (!GROUPED && D && !make_tmap_out(&td, D, (uint64_t)N, (uint64_t)M, MODE == kModeWgrad ? 4 : 2))
         return FP8Q_ERR_CUDA;
+    if (q_out && !make_tmap_out(&tq, q_out, (uint64_t)N, (uint64_t)M, 1)) return FP8Q_ERR_CUDA;
     GemmArgs a;
     a.sA = sA;
     a.sB = sB;
@@ -234,6 +240,9 @@ int launch_gemm(const uint8_t* A, const float* sA, const uint8_t* B, const float
     a.stamp = 0;
     a.units = 0;
     a.accumulate = accumulate ? 1 : 0;
+    a.s_out = s_out;
+    a.quant_out = q_out ? 1 : 0;
+    a.store_d = D ? 1 : 0;
     const int sms = sm_count();
     if (sms <= 0) return FP8Q_ERR_CUDA;
     // Grouped: at most ceil(Mtot/128) + E row tiles (each group adds at most one partial tile).
@@ -250,13 +259,13 @@ int launch_gemm(const uint8_t* A, const float* sA, const uint8_t* B, const float
             a.units = units;
             // CTAs wait on each other's partials: launch them co-resident (cooperative launch).
             return launch_kernel(gemm_blockscaled_kernel<MODE, BN, GROUPED>, dim3((unsigned)grid),
-                                 dim3(S::kThreads), S::kSmemBytes, st, true, ta, tb, td, a);
+                                 dim3(S::kThreads), S::kSmemBytes, st, true, ta, tb, td, tq, a);
         }
     }
     const int grid = (int)(tiles < sms ? tiles : sms);
     if (grid <= 0) return FP8Q_OK;
     return launch_kernel(gemm_blockscaled_kernel<MODE, BN, GROUPED>, dim3((unsigned)grid), dim3(S::kThreads),
-                         S::kSmemBytes, st, false, ta, tb, td, a);
+                         S::kSmemBytes, st, false, ta, tb, td, tq, a);
 }
 
 // Tile width: 256 whenever N allows it (measured faster on every linear-layer and MLA shape: it
@@ -460,6 +469,35 @@ int fp8_gemm_blockscaled(int mode, const uint8_t* A, const float* sA, const uint
     case FP8Q_WGRAD: return gemm_mode<kModeWgrad>(A, sA, B, sB, D, M, N, K, st, workspace, ws_bytes);
     default: return gemm_mode<kModeWgrad>(A, sA, B, sB, D, M, N, K, st, workspace, ws_bytes, true);
     }
+}
+
+int fp8_gemm_blockscaled_quant(int mode, const uint8_t* A, const float* sA, const uint8_t* B, const float* sB,
+                               void* D, uint8_t* Dq, float* Ds, int64_t M, int64_t N, int64_t K, void* workspace,
+                               size_t ws_bytes, fp8q_stream_t stream)
+{
+    if (mode != FP8Q_FPROP && mode != FP8Q_DGRAD) return FP8Q_ERR_ARG;
+    if (M < 0 || N < 0 || K < 0) return FP8Q_ERR_ARG;
+    if (N % 128 != 0 || K % 128 != 0) return FP8Q_ERR_SHAPE;
+    if (M == 0 || N == 0) return FP8Q_OK;
+    if (M >= (1ll << 31) || N >= (1ll << 31) || K >= (1ll << 31) || K == 0) return FP8Q_ERR_UNSUPPORTED;
+    if (!A || !sA || !B || !sB || !Dq || !Ds) return FP8Q_ERR_ARG;
+    if (!aligned16(A) || !aligned16(sA) || !aligned16(B) || !aligned16(sB) || !aligned16(D) || !aligned16(Dq) ||
+        !aligned16(Ds))
+        return FP8Q_ERR_ALIGN;
+    const cudaStream_t st = (cudaStream_t)stream;
+    if (choose_bn(M, N, 0) == 256) {
+        // One 256-wide tile row per promotion warp pair: each thread's 128 columns are a group.
+        if (mode == FP8Q_FPROP)
+            return launch_gemm<kModeFprop, 256, false>(A, sA, B, sB, D, nullptr, 1, M, N, K, st, workspace,
+                                                      ws_bytes, false, Dq, Ds);
+        return launch_gemm<kModeDgrad, 256, false>(A, sA, B, sB, D, nullptr, 1, M, N, K, st, workspace, ws_bytes,
+                                                  false, Dq, Ds);
+    }
+    // 128-wide tiles split a group over two warps: run the GEMM, then quantise D.
+    if (!D) return FP8Q_ERR_UNSUPPORTED;
+    const int rc = fp8_gemm_blockscaled(mode, A, sA, B, sB, D, M, N, K, workspace, ws_bytes, stream);
+    if (rc != FP8Q_OK) return rc;
+    return fp8q_act_1x128(static_cast<const uint16_t*>(D), M, N, Dq, Ds, stream);
 }
 
 int fp8_gemm_blockscaled_noalloc(int mode, const uint8_t* A, const float* sA, const uint8_t* B, const float* sB,

@@ -28,6 +28,7 @@
 #include <stdint.h>
 
 #include "ptx.cuh"
+#include "quant.cuh"
 
 namespace fp8q {
 
@@ -49,6 +50,12 @@ struct GemmArgs {
     unsigned long long stamp; // unique per launch, so flags never need resetting
     int64_t units;            // tiles * KB
     int32_t accumulate;       // Wgrad only: 1 adds the result into D (D += dY^T X), 0 overwrites D
+    // Fused 1x128 quantisation of the bf16 output (dense Fprop / Dgrad with 256-wide tiles):
+    // q_out [M][N] E4M3 codes and s_out [N/128][M] scales of bf16(D), exactly what the 1x128
+    // activation quantiser would produce from the stored D; nullptr = off.  store_d = 0 skips D.
+    float* s_out;
+    int32_t quant_out;
+    int32_t store_d;
 };
 
 // One piece of work: groups [kb0, kb1) of tile `tile`.
@@ -182,7 +189,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 template <int MODE, int BN, bool GROUPED>
 __global__ void __launch_bounds__(GemmShape<MODE, BN, GROUPED>::kThreads, 1)
 gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                        const __grid_constant__ CUtensorMap tmD, const GemmArgs args)
+                        const __grid_constant__ CUtensorMap tmD, const __grid_constant__ CUtensorMap tmQ,
+                        const GemmArgs args)
 {
     using S = GemmShape<MODE, BN, GROUPED>;
     extern __shared__ uint8_t smem_raw[];
@@ -576,9 +584,29 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                 constexpr int kSlabCols = 64 / kElt;
                 uint4* stage0 = reinterpret_cast<uint4*>(smem + S::kOffEpi) + pw * 128 * S::kEpiBufs;
                 const int wrow0 = ti.row0 + quad * 32;
+                // Fused 1x128 quantisation: this thread's kCols = 128 columns of its row are one
+                // group.  Its scale comes from the bf16-rounded outputs, as the activation
+                // quantiser would see them in D.
+                constexpr bool kCanQuant = (MODE != kModeWgrad) && !GROUPED && S::kCols == 128;
+                const bool quant = kCanQuant && args.quant_out;
+                float qinv = 0.0f;
+                if (quant) {
+                    float amax = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < S::kCols / 2; ++i) {
+                        const uint32_t h = pack_bf16x2(acc[i].x, acc[i].y);
+                        amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(h)), fabsf(bf16_hi(h))));
+                    }
+                    float qs;
+                    group_scale(amax, qs, qinv);
+                    if (row < args.M) args.s_out[(size_t)(ncol0 >> 7) * (size_t)args.M + row] = qs;
+                }
+                const bool store_d = GROUPED || MODE == kModeWgrad || args.store_d;
+                int nslab = 0;   // slabs staged so far (rotates the staging buffers)
 #pragma unroll
                 for (int sl = 0; sl < S::kCols / kSlabCols; ++sl) {
-                    uint4* stage = stage0 + (sl % S::kEpiBufs) * 128;
+                    if (!store_d) break;
+                    uint4* stage = stage0 + (nslab++ % S::kEpiBufs) * 128;
                     uint4 u[4];
 #pragma unroll
                     for (int p = 0; p < 4; ++p) {
@@ -639,6 +667,39 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                             }
                         }
                         __syncwarp();
+                    }
+                }
+                if (kCanQuant && quant) {
+                    // Codes: two 64-column slabs of E4M3 (64 bytes per row), through the same
+                    // staging buffers and a tensor map over q_out.
+#pragma unroll
+                    for (int cs = 0; cs < 2; ++cs) {
+                        uint4* stage = stage0 + (nslab++ % S::kEpiBufs) * 128;
+                        uint4 u[4];
+#pragma unroll
+                        for (int p = 0; p < 4; ++p) {
+                            uint32_t wv[4];
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                const int c = cs * 32 + p * 8 + 2 * k;   // float2 index: columns 2c, 2c+1 and 2c+2, 2c+3
+                                const uint32_t h0 = pack_bf16x2(acc[c].x, acc[c].y);
+                                const uint32_t h1 = pack_bf16x2(acc[c + 1].x, acc[c + 1].y);
+                                wv[k] = e4m3x2(__fmul_rn(bf16_lo(h0), qinv), __fmul_rn(bf16_hi(h0), qinv)) |
+                                        (e4m3x2(__fmul_rn(bf16_lo(h1), qinv), __fmul_rn(bf16_hi(h1), qinv)) << 16);
+                            }
+                            u[p] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                        }
+                        if (lane == 0) bulk_wait_group_read<S::kEpiBufs - 1>();
+                        __syncwarp();
+                        const int wsw = (lane >> 1) & 3;
+#pragma unroll
+                        for (int p = 0; p < 4; ++p) stage[lane * 4 + (p ^ wsw)] = u[p];
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&tmQ, smem_u32(stage), ncol0 + cs * 64, wrow0);
+                            bulk_commit_group();
+                        }
                     }
                 }
             }

@@ -50,6 +50,7 @@ def lib() -> ctypes.CDLL:
         "fp8q_quant_forward": [P, I64, I64, P, P, P, P, P, I64, P, P, P, P],
         "fp8q_weight_128x128": [P, I64, I64, P, P, P, P],
         "fp8_gemm_blockscaled": [I, P, P, P, P, P, I64, I64, I64, P, ctypes.c_size_t, P],
+        "fp8_gemm_blockscaled_quant": [I, P, P, P, P, P, P, P, I64, I64, I64, P, ctypes.c_size_t, P],
         "fp8_grouped_gemm_blockscaled": [P, P, P, P, P, I32, I64, I64, I64, P, P],
         "fp8q_device_status": [P, ctypes.POINTER(I)],
     }.items():
@@ -231,6 +232,37 @@ def gemm_blockscaled(mode: int, A: torch.Tensor, sA: torch.Tensor, B: torch.Tens
            lib().fp8_gemm_blockscaled(int(mode), _p(A), _p(sA), _p(B), _p(sB), _p(out), M, N, K,
                                       ws_ptr, ws_bytes, _stream(A.device)))
     return out
+
+
+def gemm_blockscaled_quant(mode: int, A: torch.Tensor, sA: torch.Tensor, B: torch.Tensor,
+                           sB: torch.Tensor, out: torch.Tensor | None = None, q: torch.Tensor | None = None,
+                           s: torch.Tensor | None = None, store_out: bool = True,
+                           workspace: torch.Tensor | None = None):
+    """FPROP / DGRAD that also returns the 1x128 E4M3 codes and scales of its bf16 output (as
+    act_1x128 would compute them from it).  Returns (D or None, q[M,N] uint8, s[N/128, M] fp32);
+    store_out=False skips writing the bf16 D."""
+    if mode not in (FPROP, DGRAD):
+        raise ValueError("the fused output quantisation exists for FPROP and DGRAD")
+    _require(A, "A", torch.uint8, 2)
+    _require(B, "B", torch.uint8, 2)
+    _require(sA, "sA", torch.float32, 2)
+    _require(sB, "sB", torch.float32, 2)
+    M, K = A.shape
+    N = B.shape[1] if mode == DGRAD else B.shape[0]
+    dev = A.device
+    if store_out:
+        out = _out(out, (M, N), torch.bfloat16, dev, "out")
+    else:
+        out = None
+    q = _out(q, (M, N), torch.uint8, dev, "q")
+    s = _out(s, (N // 128, M), torch.float32, dev, "s")
+    if workspace is None:
+        workspace = gemm_workspace(mode, M, N, K, dev)
+    ws_ptr, ws_bytes = (None, 0) if workspace is None else (_p(workspace), workspace.numel())
+    _check("fp8_gemm_blockscaled_quant",
+           lib().fp8_gemm_blockscaled_quant(int(mode), _p(A), _p(sA), _p(B), _p(sB), _p(out), _p(q), _p(s),
+                                            M, N, K, ws_ptr, ws_bytes, _stream(dev)))
+    return out, q, s
 
 
 def grouped_gemm_blockscaled(A: torch.Tensor, sA: torch.Tensor, B: torch.Tensor,

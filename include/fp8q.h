@@ -177,6 +177,22 @@ FP8Q_API int fp8_gemm_blockscaled(int mode, const uint8_t* A, const float* sA, c
 FP8Q_API size_t fp8q_gemm_workspace_size(int mode, int64_t M, int64_t N, int64_t K);
 
 /*
+ * Fprop or Dgrad (mode FP8Q_FPROP / FP8Q_DGRAD, arguments as fp8_gemm_blockscaled) that also
+ * quantises its output for the next GEMM: the 1x128 tile-wise E4M3 codes and scales of the bf16
+ * output, written from the epilogue while the output tile is still in registers.
+ *   D  : [M, N] bf16, or NULL to skip storing the bf16 output (then N % 256 == 0 is required)
+ *   Dq : [M, N] E4M3 codes,  Ds : [N/128, M] fp32 scales -- bit-identical to
+ *        fp8q_act_1x128(D) applied to the bf16 output this call computes.
+ * With N % 256 == 0 (256-wide tiles: each promotion thread holds one row's 128-column group) the
+ * quantisation runs in the GEMM epilogue; otherwise the call runs the GEMM and then
+ * fp8q_act_1x128 on D (D required).  K > 0; other requirements and errors as
+ * fp8_gemm_blockscaled.
+ */
+FP8Q_API int fp8_gemm_blockscaled_quant(int mode, const uint8_t* A, const float* sA, const uint8_t* B,
+                                        const float* sB, void* D, uint8_t* Dq, float* Ds, int64_t M, int64_t N,
+                                        int64_t K, void* workspace, size_t ws_bytes, fp8q_stream_t stream);
+
+/*
  * fp8_gemm_blockscaled without a workspace argument, for callers that may not allocate device
  * memory themselves: a plugin running inside a host framework that owns the device memory pool
  * and gives its kernels only their inputs and outputs, or a latency-critical path that cannot

@@ -121,6 +121,19 @@ def test_gemm_host_checks(L):
     assert L.fp8q_gemm_workspace_size(0, 4096, 2048, 128) == 0
 
 
+def test_gemm_quant_host_checks(L):
+    s = None
+    g = L.fp8_gemm_blockscaled_quant
+    ab = (P(FAKE), P(FAKE), P(FAKE), P(FAKE))
+    ws = (None, 0, s)
+    assert g(2, *ab, P(FAKE), P(FAKE), P(FAKE), 128, 256, 128, *ws) == ERR_ARG          # Wgrad: no
+    assert g(0, *ab, P(FAKE), None, P(FAKE), 128, 256, 128, *ws) == ERR_ARG              # Dq missing
+    assert g(0, *ab, P(FAKE), P(FAKE), P(FAKE), 128, 100, 128, *ws) == ERR_SHAPE
+    assert g(0, *ab, P(FAKE), P(FAKE), P(FAKE), 128, 256, 0, *ws) == ERR_UNSUPPORTED     # K = 0
+    assert g(0, *ab, P(FAKE), P(FAKE), P(MISALIGNED), 128, 256, 128, *ws) == ERR_ALIGN
+    assert g(1, *ab, P(FAKE), P(FAKE), P(FAKE), 0, 256, 128, *ws) == OK                  # no rows
+
+
 def test_grouped_host_checks(L):
     s = None
     g = L.fp8_grouped_gemm_blockscaled

@@ -188,6 +188,60 @@ def test_wgrad_accumulate_rejects_missing_out():
         ops.gemm_blockscaled(WGRAD_ACC, *(torch.zeros(1, device="cuda"),) * 4)
 
 
+def check_gemm_quant(mode, A, sA, B, sB, what, monkeypatch=None, bn=None):
+    """D within the GEMM tolerance, and (q, s) bit-exact against the oracle's 1x128 quantiser
+    applied to the bf16 D this call returned; the same call without storing D gives the same
+    codes and scales."""
+    if bn is not None:
+        set_config(monkeypatch, bn)
+    args = (u8_dev(A), f32_dev(sA), u8_dev(B), f32_dev(sB))
+    D, q, s = ops.gemm_blockscaled_quant(mode, *args)
+    torch.cuda.synchronize()
+    assert ops.device_status() == ops.DEV_OK
+    d_bits = D.view(torch.int16).cpu().numpy().view(np.uint16)
+    ref, S = oracle.gemm(mode, A, sA, B, sB)
+    check_gemm(host(D).astype(np.float64), ref, S, what)
+    oq, os_ = oracle.quant_1x128(d_bits)
+    assert np.array_equal(host(q), oq), f"{what}: codes differ from the 1x128 quantiser of D"
+    assert np.array_equal(host(s).view(np.uint32), os_.view(np.uint32)), f"{what}: scales differ"
+    if B.shape[1 if mode == DGRAD else 0] % 256 == 0 and bn in (None, "n256-dp", "n256-sk"):
+        _, q2, s2 = ops.gemm_blockscaled_quant(mode, *args, store_out=False)
+        torch.cuda.synchronize()
+        assert torch.equal(q2, q) and torch.equal(s2, s), f"{what}: store_out=False changed the codes"
+
+
+@pytest.mark.parametrize("bn", list(CONFIGS))
+@pytest.mark.parametrize("M,N,K", [(256, 512, 512), (300, 768, 1024)])
+def test_fprop_fused_output_quant(M, N, K, bn, monkeypatch):
+    X = synth.activations_entry_outliers(M, K, seed=M + 5)
+    W = synth.weights(N, K, seed=N + 6)
+    xq, xs = oracle.quant_1x128(X)
+    wq, ws, _ = oracle.quant_128x128(W)
+    check_gemm_quant(FPROP, xq, xs, wq, ws, f"fprop+quant {M}x{N}x{K}", monkeypatch, bn)
+
+
+@pytest.mark.parametrize("bn", list(CONFIGS))
+def test_dgrad_fused_output_quant(bn, monkeypatch):
+    M, N, K = 384, 640, 512                      # N = 640: 256-wide tiles do not fit (fallback path)
+    dY = synth.output_grad(M, K, seed=81)
+    W = synth.weights(K, N, seed=82)
+    gq, gs = oracle.quant_1x128(dY)
+    wq, ws, _ = oracle.quant_128x128(W)
+    check_gemm_quant(DGRAD, gq, gs, wq, ws, f"dgrad+quant {M}x{N}x{K}", monkeypatch, bn)
+
+
+def test_full_fprop_fused_output_quant():
+    q = quantised_layer()
+    (xq, xs), (wq, ws) = q["X"], q["W"]
+    args = (u8_dev(xq), f32_dev(xs), u8_dev(wq), f32_dev(ws))
+    D, qd, sd = ops.gemm_blockscaled_quant(FPROP, *args)
+    plain = ops.gemm_blockscaled(FPROP, *args)
+    torch.cuda.synchronize()
+    assert torch.equal(D, plain), "the fused epilogue changed the bf16 output"
+    oq, os_ = oracle.quant_1x128(D.view(torch.int16).cpu().numpy().view(np.uint16))
+    assert np.array_equal(host(qd), oq) and np.array_equal(host(sd).view(np.uint32), os_.view(np.uint32))
+
+
 # ------------------------------------------------------------------------------------------ #
 # Tolerance cases, full outputs
 # ------------------------------------------------------------------------------------------ #
