@@ -294,6 +294,30 @@ def run_ours(args, rank, world, dist):
     for s in range(bsteps):
         for i, name in enumerate(OPS):
             per_op[name].append(bevs[s][i].elapsed_time(bevs[s][i + 1]))
+
+    # Not part of the step: Fprop with the next layer's 1x128 quantisation of Y fused into its
+    # epilogue, against Fprop followed by the separate quantiser.
+    yq = torch.empty((T_TOK, C_OUT), dtype=torch.uint8, device=dev)
+    ys = torch.empty((C_OUT // 128, T_TOK), dtype=torch.float32, device=dev)
+    fused_runs = {
+        "fprop": lambda: ops.gemm_blockscaled(ops.FPROP, b["Xq"], b["sX"], b["Wq"], b["sW"], b["Y"]),
+        "fprop_then_act_1x128_Y": lambda: (ops.gemm_blockscaled(ops.FPROP, b["Xq"], b["sX"], b["Wq"], b["sW"], b["Y"]),
+                                           ops.act_1x128(b["Y"], yq, ys)),
+        "fprop_fused_quant_Y": lambda: ops.gemm_blockscaled_quant(ops.FPROP, b["Xq"], b["sX"], b["Wq"], b["sW"],
+                                                                  b["Y"], yq, ys),
+    }
+    fused_ms = {}
+    for name, f in fused_runs.items():
+        ts = []
+        for _ in range(10):
+            flush_l2()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            f()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        fused_ms[name] = round(statistics.median(ts[2:]), 5)
     sum_step_ms = float(sum(step_ms))
     total_ms = start.elapsed_time(end)
     sum_step_ms = max_over_ranks(sum_step_ms, dist, dev)
@@ -354,8 +378,8 @@ def run_ours(args, rank, world, dist):
                        "(nominal dense FP8/BF16 ratio)",
         "traffic": (traffic or {}).get("gemm_bytes_per_launch"),
     }
-    q_ms = sum(statistics.mean(per_op[n]) for n in OPS if n.startswith(("act", "weight")))
-    q_bytes = sum(work[n][1] for n in OPS if n.startswith(("act", "weight")))
+    q_ms = sum(statistics.mean(per_op[n]) for n in OPS if n.startswith(("act", "weight", "quant")))
+    q_bytes = sum(work[n][1] for n in OPS if n.startswith(("act", "weight", "quant")))
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
@@ -369,6 +393,7 @@ def run_ours(args, rank, world, dist):
                        "frac_hbm": round(q_bytes / (q_ms * 1e-3) / 1e9 / hbm, 4),
                        "hbm_peak_gbs": hbm, "peak_source": peak_kind},
         "kernels": kernels,
+        "fused_output_quant_ms": fused_ms,
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "steps": len(e2e_ms)},
         "gpu_launches": len(launches) * args.steps,
