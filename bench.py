@@ -563,6 +563,26 @@ def run_moe(args, rank, world, dist):
             f()
             bevs[s_][i + 1].record()
     torch.cuda.synchronize()
+    # Not part of the step: the experts' input gradient, grouped Dgrad dX = dY W_e over the same
+    # rows, with the same (forward) expert weights and a seeded dY quantised on the device.
+    dy = (1e-3 * torch.randn((mtot, MOE_N), device=dev, generator=g)).to(torch.bfloat16)
+    dyq = torch.empty((mtot, MOE_N), dtype=torch.uint8, device=dev)
+    dys = torch.empty((MOE_N // 128, mtot), dtype=torch.float32, device=dev)
+    ops.act_1x128(dy, dyq, dys)
+    dx = torch.empty((mtot, MOE_K), dtype=torch.bfloat16, device=dev)
+    dts = []
+    for _ in range(8):
+        flush_l2()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        ops.grouped_gemm_blockscaled_dgrad(dyq, dys, wq.view(MOE_E, MOE_N, MOE_K),
+                                           sw.view(MOE_E, MOE_N // 128, MOE_K // 128), offsets, dx)
+        e1.record()
+        torch.cuda.synchronize()
+        dts.append(e0.elapsed_time(e1))
+    if ops.device_status(dev) != ops.DEV_OK:
+        raise RuntimeError("device status after the grouped Dgrad")
+    dgrad_ms = statistics.median(dts[2:])
     peaks, peak_kind = load_peaks()
     fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
     kernels = {}
@@ -589,6 +609,9 @@ def run_moe(args, rank, world, dist):
                      "unit": "TFLOP/s", "frac": round(flop / (g_ms * 1e-3) / 1e12 / fp8_peak, 4),
                      "peak_source": f"{peak_kind} bf16 burst x {FP8_OVER_BF16}", "traffic": None},
         "kernels": kernels,
+        "grouped_dgrad": {"ms": round(dgrad_ms, 4), "TFLOP/s": round(flop / (dgrad_ms * 1e-3) / 1e12, 1),
+                          "frac_fp8_peak": round(flop / (dgrad_ms * 1e-3) / 1e12 / fp8_peak, 4),
+                          "note": "dX [rows, 7168] = dY [rows, 2048] W_e, not part of the step"},
         "e2e": None,
         "e2e_note": "not measured for this secondary workload (the expert weights alone are 7.5 GB of H2D per step)",
         "gpu_launches": len(launches) * args.steps,

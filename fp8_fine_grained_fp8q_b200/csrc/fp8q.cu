@@ -215,7 +215,8 @@ int launch_gemm(const uint8_t* A, const float* sA, const uint8_t* B, const float
     CUtensorMap ta, tb;
     if (!make_tmap_u8(&ta, A, (uint64_t)K, (uint64_t)M, 128, 128)) return FP8Q_ERR_CUDA;
     if (MODE == kModeDgrad) {
-        if (!make_tmap_u8(&tb, B, (uint64_t)N, (uint64_t)K, 128, 128)) return FP8Q_ERR_CUDA;
+        const uint64_t krows = GROUPED ? (uint64_t)E * (uint64_t)K : (uint64_t)K;
+        if (!make_tmap_u8(&tb, B, (uint64_t)N, krows, 128, 128)) return FP8Q_ERR_CUDA;
     } else {
         const uint64_t rows = GROUPED ? (uint64_t)E * (uint64_t)N : (uint64_t)N;
         if (!make_tmap_u8(&tb, B, (uint64_t)K, rows, 128, BN)) return FP8Q_ERR_CUDA;
@@ -534,6 +535,27 @@ int fp8_grouped_gemm_blockscaled(const uint8_t* A, const float* sA, const uint8_
     if (choose_bn(Mtot, N, E) == 256)
         return launch_gemm<kModeFprop, 256, true>(A, sA, B, sB, D, offsets, E, Mtot, N, K, st);
     return launch_gemm<kModeFprop, 128, true>(A, sA, B, sB, D, offsets, E, Mtot, N, K, st);
+}
+
+int fp8_grouped_gemm_blockscaled_dgrad(const uint8_t* A, const float* sA, const uint8_t* B, const float* sB,
+                                       const int32_t* offsets, int32_t E, int64_t Mtot, int64_t N, int64_t K,
+                                       uint16_t* D, fp8q_stream_t stream)
+{
+    if (E < 1 || Mtot < 0 || N < 0 || K < 0) return FP8Q_ERR_ARG;
+    if (E > 1024) return FP8Q_ERR_UNSUPPORTED;
+    if (N % 128 != 0 || K % 128 != 0) return FP8Q_ERR_SHAPE;
+    if (Mtot == 0 || N == 0) return FP8Q_OK;
+    if (Mtot >= (1ll << 31) || N >= (1ll << 31) || (int64_t)E * K >= (1ll << 31)) return FP8Q_ERR_UNSUPPORTED;
+    if (!A || !sA || !B || !sB || !D || !offsets) return FP8Q_ERR_ARG;
+    if (!aligned16(A) || !aligned16(sA) || !aligned16(B) || !aligned16(sB) || !aligned16(D)) return FP8Q_ERR_ALIGN;
+    if ((reinterpret_cast<uintptr_t>(offsets) & 3u) != 0) return FP8Q_ERR_ALIGN;
+    const cudaStream_t st = (cudaStream_t)stream;
+    if (K == 0) {
+        return cudaMemsetAsync(D, 0, (size_t)Mtot * (size_t)N * 2u, st) == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+    }
+    if (choose_bn(Mtot, N, E) == 256)
+        return launch_gemm<kModeDgrad, 256, true>(A, sA, B, sB, D, offsets, E, Mtot, N, K, st);
+    return launch_gemm<kModeDgrad, 128, true>(A, sA, B, sB, D, offsets, E, Mtot, N, K, st);
 }
 
 int fp8q_selftest_wait_timeout(uint64_t limit_ns, fp8q_stream_t stream)

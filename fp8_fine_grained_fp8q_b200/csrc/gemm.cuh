@@ -36,7 +36,7 @@ enum { kModeFprop = 0, kModeDgrad = 1, kModeWgrad = 2 };
 
 struct GemmArgs {
     const float* sA;          // [KB][M]
-    const float* sB;          // Fprop [N/128][KB] (x E if grouped); Dgrad [KB][N/128]; Wgrad [KB][N]
+    const float* sB;          // Fprop [N/128][KB], Dgrad [KB][N/128] (each x E if grouped); Wgrad [KB][N]
     void* D;                  // [M][N], bf16 (Fprop / Dgrad) or fp32 (Wgrad)
     const int32_t* offsets;   // grouped only: device [E+1]
     int32_t E;                // number of groups (1 unless grouped)
@@ -311,8 +311,9 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                     tma_load_2d(sa, &tmA, kb * 128, ti.row0, full_bar(stage));
                     if (MODE == kModeDgrad) {
 #pragma unroll
-                        for (int h = 0; h < BN / 128; ++h)
-                            tma_load_2d(sb + h * 16384, &tmB, ti.n0 + h * 128, kb * 128, full_bar(stage));
+                        for (int h = 0; h < BN / 128; ++h)   // grouped: expert e's K rows start at e * K
+                            tma_load_2d(sb + h * 16384, &tmB, ti.n0 + h * 128, (GROUPED ? ti.e * KB * 128 : 0) + kb * 128,
+                                        full_bar(stage));
                     } else {
                         tma_load_2d(sb, &tmB, kb * 128, brow, full_bar(stage));
                     }
@@ -424,7 +425,7 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                 sb_ptr = args.sB + (size_t)ti.e * (size_t)(args.N >> 7) * KB + (size_t)(ncol0 >> 7) * KB;
                 sb_step = 1;
             } else if (MODE == kModeDgrad) {
-                sb_ptr = args.sB + (ncol0 >> 7);
+                sb_ptr = args.sB + (size_t)ti.e * (size_t)KB * (size_t)(args.N >> 7) + (ncol0 >> 7);
                 sb_step = (size_t)(args.N >> 7);
             }
 #pragma unroll

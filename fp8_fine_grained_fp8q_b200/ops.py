@@ -52,6 +52,7 @@ def lib() -> ctypes.CDLL:
         "fp8_gemm_blockscaled": [I, P, P, P, P, P, I64, I64, I64, P, ctypes.c_size_t, P],
         "fp8_gemm_blockscaled_quant": [I, P, P, P, P, P, P, P, I64, I64, I64, P, ctypes.c_size_t, P],
         "fp8_grouped_gemm_blockscaled": [P, P, P, P, P, I32, I64, I64, I64, P, P],
+        "fp8_grouped_gemm_blockscaled_dgrad": [P, P, P, P, P, I32, I64, I64, I64, P, P],
         "fp8q_device_status": [P, ctypes.POINTER(I)],
     }.items():
         fn = getattr(L, name)
@@ -285,6 +286,30 @@ def grouped_gemm_blockscaled(A: torch.Tensor, sA: torch.Tensor, B: torch.Tensor,
     _check("fp8_grouped_gemm_blockscaled",
            lib().fp8_grouped_gemm_blockscaled(_p(A), _p(sA), _p(B), _p(sB), _p(offsets), E, Mtot,
                                               N, K, _p(out), _stream(A.device)))
+    return out
+
+
+def grouped_gemm_blockscaled_dgrad(A: torch.Tensor, sA: torch.Tensor, B: torch.Tensor,
+                                   sB: torch.Tensor, offsets: torch.Tensor,
+                                   out: torch.Tensor | None = None):
+    """Grouped Dgrad: A = dY codes [Mtot,K], sA[K/128,Mtot], B = forward expert weights
+    [E,K,N] (out = K, in = N), sB[E,K/128,N/128], offsets int32[E+1] on the device.
+    Returns dX[Mtot,N] bf16."""
+    _require(A, "A", torch.uint8, 2)
+    _require(B, "B", torch.uint8, 3)
+    _require(sA, "sA", torch.float32, 2)
+    _require(sB, "sB", torch.float32, 3)
+    _require(offsets, "offsets", torch.int32, 1)
+    Mtot, K = A.shape
+    E, Kb, N = B.shape
+    if Kb != K:
+        raise ValueError("inner dimensions differ")
+    if offsets.numel() != E + 1:
+        raise ValueError("offsets must have E+1 entries")
+    out = _out(out, (Mtot, N), torch.bfloat16, A.device, "out")
+    _check("fp8_grouped_gemm_blockscaled_dgrad",
+           lib().fp8_grouped_gemm_blockscaled_dgrad(_p(A), _p(sA), _p(B), _p(sB), _p(offsets), E, Mtot,
+                                                    N, K, _p(out), _stream(A.device)))
     return out
 
 

@@ -233,6 +233,21 @@ FP8Q_API int fp8_grouped_gemm_blockscaled(const uint8_t* A, const float* sA, con
                                  fp8q_stream_t stream);
 
 /*
+ * Grouped Dgrad over the same ragged row groups: dX_e = dY_e W_e for every expert, the input
+ * gradient of the grouped Fprop ([REPOST] paragraph 2: Dgrad in FP8; 256 routed experts,
+ * [SUMMARY]).  The expert weights are the forward ones, used transposed without requantisation:
+ *   A  : [Mtot, K] codes of dY (K = the experts' output width), sA : [K/128, Mtot] (1x128)
+ *   B  : [E, K, N] codes -- expert e's forward weight [out = K, in = N] -- and
+ *   sB : [E, K/128, N/128] its forward 128x128 block scales
+ *   offsets : as fp8_grouped_gemm_blockscaled (validated on the device the same way)
+ *   D  : [Mtot, N] bf16.
+ * Requirements and errors as fp8_grouped_gemm_blockscaled, with E * K < 2^31.
+ */
+FP8Q_API int fp8_grouped_gemm_blockscaled_dgrad(const uint8_t* A, const float* sA, const uint8_t* B,
+                                                const float* sB, const int32_t* offsets, int32_t E, int64_t Mtot,
+                                                int64_t N, int64_t K, uint16_t* D, fp8q_stream_t stream);
+
+/*
  * Synchronise `stream`, then read and clear the device status word of the current device.
  * *out receives FP8Q_DEV_OK or the first error latched since the last call.  Returns FP8Q_OK,
  * FP8Q_ERR_ARG (out == NULL) or FP8Q_ERR_CUDA.

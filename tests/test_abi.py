@@ -146,6 +146,18 @@ def test_grouped_host_checks(L):
     assert g(P(FAKE), P(FAKE), P(FAKE), P(FAKE), None, 4, 128, 128, 128, P(FAKE), s) == ERR_ARG
 
 
+def test_grouped_dgrad_host_checks(L):
+    s = None
+    g = L.fp8_grouped_gemm_blockscaled_dgrad
+    a = (P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE))
+    assert g(*a, 0, 128, 128, 128, P(FAKE), s) == ERR_ARG
+    assert g(*a, 2000, 128, 128, 128, P(FAKE), s) == ERR_UNSUPPORTED
+    assert g(*a, 4, 128, 128, 100, P(FAKE), s) == ERR_SHAPE
+    assert g(*a, 4, 0, 128, 128, P(FAKE), s) == OK
+    assert g(P(FAKE), P(FAKE), P(FAKE), P(FAKE), None, 4, 128, 128, 128, P(FAKE), s) == ERR_ARG
+    assert g(P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE + 2), 4, 128, 128, 128, P(FAKE), s) == ERR_ALIGN
+
+
 def test_selftest_and_status_arg_checks(L):
     assert L.fp8q_selftest_wait_timeout(0, None) == ERR_ARG
     assert L.fp8q_selftest_wait_timeout(3_000_000_000, None) == ERR_ARG

@@ -1,4 +1,5 @@
-"""GPU grouped (MoE expert) block-scaled FP8 Fprop vs the oracle, and the device-side checks.
+"""GPU grouped (MoE expert) block-scaled FP8 Fprop and Dgrad vs the oracle, and the device-side
+checks.
 
 Row groups come from the seeded Zipf-skewed top-8 routing (some experts empty).  Small cases
 compare every output; the full-size case (8192 tokens x top-8 over 256 experts, N = 2048,
@@ -54,6 +55,52 @@ def test_grouped_small_all_entries(counts, bn, monkeypatch):
     ms, ns = np.meshgrid(np.arange(Mtot), np.arange(N), indexing="ij")
     ref, S = oracle.grouped_entries(aq, as_, bq, bs, off, ms.reshape(-1), ns.reshape(-1))
     check_gemm(got, ref.reshape(Mtot, N), S.reshape(Mtot, N), f"grouped {counts}")
+
+
+def dgrad_problem(counts, Nin, Kout, seed):
+    """dY rows grouped by expert and the experts' forward weights W_e [Kout, Nin] (128x128)."""
+    counts = np.asarray(counts)
+    E = counts.size
+    off = np.zeros(E + 1, dtype=np.int32)
+    off[1:] = np.cumsum(counts)
+    Mtot = int(off[-1])
+    dY = synth.output_grad(max(Mtot, 1), Kout, seed=seed)[:Mtot]
+    gq, gs = oracle.quant_1x128(dY)
+    wq = np.empty((E, Kout, Nin), dtype=np.uint8)
+    ws = np.empty((E, Kout // 128, Nin // 128), dtype=np.float32)
+    for e in range(E):
+        wq[e], ws[e], _ = oracle.quant_128x128(synth.weights(Kout, Nin, seed=seed * 37 + e))
+    return gq, gs, wq, ws, off
+
+
+@pytest.mark.parametrize("bn", [128, 256])
+@pytest.mark.parametrize("counts", [[0, 1, 130, 0, 255, 64], [128], [5, 0, 300]])
+def test_grouped_dgrad_small_all_entries(counts, bn, monkeypatch):
+    Nin, Kout = 512, 256
+    monkeypatch.setenv("FP8Q_GEMM_BN", str(bn))
+    gq, gs, wq, ws, off = dgrad_problem(counts, Nin, Kout, seed=len(counts) * 7 + sum(counts))
+    out = torch.full((gq.shape[0], Nin), float("nan"), dtype=torch.bfloat16, device="cuda")
+    ops.grouped_gemm_blockscaled_dgrad(u8_dev(gq), f32_dev(gs), u8_dev(wq), f32_dev(ws),
+                                       torch.from_numpy(off).cuda(), out=out)
+    assert ops.device_status() == ops.DEV_OK
+    got = host(out)
+    for e in range(len(counts)):
+        r0, r1 = int(off[e]), int(off[e + 1])
+        if r1 == r0:
+            continue
+        ref, S = oracle.gemm(ops.DGRAD, gq[r0:r1], np.ascontiguousarray(gs[:, r0:r1]), wq[e], ws[e])
+        check_gemm(got[r0:r1], ref, S, f"grouped dgrad expert {e} ({r1 - r0} rows)")
+
+
+def test_grouped_dgrad_bad_offsets_are_reported():
+    gq, gs, wq, ws, off = dgrad_problem([128, 128], 256, 128, seed=5)
+    bad = off.copy()
+    bad[1], bad[2] = 200, 300          # the last offset (300) is not Mtot (256)
+    out = torch.full((gq.shape[0], 256), 7.0, dtype=torch.bfloat16, device="cuda")
+    ops.grouped_gemm_blockscaled_dgrad(u8_dev(gq), f32_dev(gs), u8_dev(wq), f32_dev(ws),
+                                       torch.from_numpy(bad).cuda(), out=out)
+    assert ops.device_status() == ops.DEV_BAD_OFFSETS
+    assert bool((out == 7.0).all()), "nothing may be written for malformed offsets"
 
 
 @pytest.mark.parametrize("bad", ["nonzero_start", "decreasing", "wrong_total"])
