@@ -23,7 +23,8 @@ What it computes, from the pages on the DeepSeek-V3 Technical Report (arXiv 2412
 Readings the pages leave open (OCP E4M3FN, round-to-nearest-even with saturation at 448,
 max-abs scaling with an amax floor of 2^-100) are stated in ``fp8q_oracle.c``.
 
-The arithmetic lives in ``fp8q_oracle.c``; this module only marshals numpy arrays.
+The arithmetic lives in ``fp8q_oracle.c``; this module only marshals numpy arrays (and, for the
+expert-grouped Wgrad operands, pads each expert's rows before calling it).
 """
 from __future__ import annotations
 
@@ -209,3 +210,42 @@ def grouped_entries(A, sA, B, sB, offsets, ms, ns):
     _load().oracle_grouped_entries(_ptr(A), _ptr(sA), _ptr(B), _ptr(sB), _ptr(off), E, Mtot,
                                    N, K, _ptr(ms), _ptr(ns), ms.size, _ptr(out), _ptr(sabs))
     return out, sabs
+
+
+def ragged_group_prefix(offsets) -> np.ndarray:
+    """P[e] = sum over e' < e of ceil(n_e' / 128): expert e's first 128-token group in the
+    padded token axis of the grouped Wgrad operands (P[E] groups in all)."""
+    off = np.asarray(offsets, dtype=np.int64)
+    n = off[1:] - off[:-1]
+    P = np.zeros(off.size, dtype=np.int64)
+    np.cumsum((n + 127) // 128, out=P[1:])
+    return P
+
+
+def quant_128x1_t_ragged(x_bits: np.ndarray, offsets):
+    """128x1 groups along each expert's own tokens, for the grouped Wgrad dW_e = dY_e^T X_e.
+
+    x[Mtot, C] bf16 bits with rows ordered by expert (rows offsets[e] .. offsets[e+1]-1 are
+    expert e's).  Reading (the pages fix only that the groups run along the GEMM's inner, i.e.
+    token, dimension -- repost paragraph 4): an expert's groups start at its first token; its last
+    group holds the n_e mod 128 remaining tokens and takes its max-abs over those.  That is the
+    plain 128x1 quantiser on the expert's rows zero-padded to a multiple of 128 (a zero changes
+    neither the max-abs nor a dot product), which is how it is computed here.
+    Returns qt[C, 128*P[E]] (expert e's tokens at columns 128*P[e] .., zero codes in its padding)
+    and s[P[E], C]."""
+    off = np.asarray(offsets, dtype=np.int64)
+    C = x_bits.shape[1]
+    P = ragged_group_prefix(off)
+    qt = np.zeros((C, 128 * int(P[-1])), dtype=np.uint8)
+    s = np.empty((int(P[-1]), C), dtype=np.float32)
+    for e in range(off.size - 1):
+        n = int(off[e + 1] - off[e])
+        if n == 0:
+            continue
+        g = int(P[e + 1] - P[e])
+        block = np.zeros((128 * g, C), dtype=x_bits.dtype)
+        block[:n] = x_bits[off[e]:off[e + 1]]
+        q, se = quant_128x1_t(block)
+        qt[:, 128 * int(P[e]):128 * int(P[e + 1])] = q
+        s[int(P[e]):int(P[e + 1])] = se
+    return qt, s

@@ -103,6 +103,37 @@ def test_grouped_dgrad_bad_offsets_are_reported():
     assert bool((out == 7.0).all()), "nothing may be written for malformed offsets"
 
 
+@pytest.mark.parametrize("dgrad", [False, True])
+def test_grouped_at_the_expert_limit(dgrad):
+    # 1024 experts (the most the kernels accept), most of them empty or tiny: every row of the
+    # non-empty experts is checked, and each expert's tile list is only its own rows.
+    E, N, K = 1024, 256, 256
+    g = np.random.Generator(np.random.PCG64(1024))
+    counts = np.where(g.random(E) < 0.8, 0, g.integers(1, 200, size=E))
+    counts[[0, E - 1]] = [3, 129]
+    off = np.zeros(E + 1, dtype=np.int32)
+    off[1:] = np.cumsum(counts)
+    Mtot = int(off[-1])
+    pool_w = [oracle.quant_128x128(synth.weights(N, K, seed=900 + p)) for p in range(4)]
+    bq = np.stack([pool_w[e % 4][0] for e in range(E)])
+    bs = np.stack([pool_w[e % 4][1] * np.float32(1 + (e % 7) / 8) for e in range(E)]).astype(np.float32)
+    A = synth.activations_channel_outliers(Mtot, K, seed=1025)
+    aq, as_ = oracle.quant_1x128(A)
+    out = torch.full((Mtot, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    offs = torch.from_numpy(off).cuda()
+    if dgrad:
+        ops.grouped_gemm_blockscaled_dgrad(u8_dev(aq), f32_dev(as_), u8_dev(bq), f32_dev(bs), offs, out=out)
+    else:
+        ops.grouped_gemm_blockscaled(u8_dev(aq), f32_dev(as_), u8_dev(bq), f32_dev(bs), offs, out=out)
+    assert ops.device_status() == ops.DEV_OK
+    got = host(out)
+    mode = ops.DGRAD if dgrad else ops.FPROP
+    for e in np.flatnonzero(counts):
+        r0, r1 = int(off[e]), int(off[e + 1])
+        ref, S = oracle.gemm(mode, aq[r0:r1], np.ascontiguousarray(as_[:, r0:r1]), bq[e], bs[e])
+        check_gemm(got[r0:r1], ref, S, f"expert {e} of {E} ({r1 - r0} rows, {'dgrad' if dgrad else 'fprop'})")
+
+
 @pytest.mark.parametrize("bad", ["nonzero_start", "decreasing", "wrong_total"])
 def test_grouped_bad_offsets_are_reported_and_nothing_written(bad):
     N, K = 128, 256
