@@ -583,6 +583,32 @@ def run_moe(args, rank, world, dist):
     if ops.device_status(dev) != ops.DEV_OK:
         raise RuntimeError("device status after the grouped Dgrad")
     dgrad_ms = statistics.median(dts[2:])
+    # Not part of the step either: the experts' weight gradients, dW_e = dY_e^T X_e over each
+    # expert's own tokens (ragged 128x1 quantisation of dY and X, then the K-grouped GEMM).
+    dw = torch.empty((MOE_E, MOE_N, MOE_K), dtype=torch.float32, device=dev)
+    kcap = ops.ragged_capacity(mtot, MOE_E)
+    dyt = torch.empty((MOE_N, kcap), dtype=torch.uint8, device=dev)
+    sdyt = torch.empty((kcap // 128, MOE_N), dtype=torch.float32, device=dev)
+    xt = torch.empty((MOE_K, kcap), dtype=torch.uint8, device=dev)
+    sxt = torch.empty((kcap // 128, MOE_K), dtype=torch.float32, device=dev)
+    wts, qts = [], []
+    for _ in range(6):
+        flush_l2()
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record()
+        ops.act_128x1_transposed_ragged(dy, offsets, kcap, dyt, sdyt)
+        ops.act_128x1_transposed_ragged(xg, offsets, kcap, xt, sxt)
+        e1.record()
+        ops.grouped_gemm_blockscaled_wgrad(dyt, sdyt, xt, sxt, offsets, mtot, dw)
+        e2.record()
+        torch.cuda.synchronize()
+        qts.append(e0.elapsed_time(e1))
+        wts.append(e1.elapsed_time(e2))
+    if ops.device_status(dev) != ops.DEV_OK:
+        raise RuntimeError("device status after the grouped Wgrad")
+    del dw
+    wgrad_ms, rq_ms = statistics.median(wts[2:]), statistics.median(qts[2:])
+    rq_bytes = mtot * (MOE_N + MOE_K) * QB_1x128
     peaks, peak_kind = load_peaks()
     fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
     kernels = {}
@@ -612,6 +638,13 @@ def run_moe(args, rank, world, dist):
         "grouped_dgrad": {"ms": round(dgrad_ms, 4), "TFLOP/s": round(flop / (dgrad_ms * 1e-3) / 1e12, 1),
                           "frac_fp8_peak": round(flop / (dgrad_ms * 1e-3) / 1e12 / fp8_peak, 4),
                           "note": "dX [rows, 7168] = dY [rows, 2048] W_e, not part of the step"},
+        "grouped_wgrad": {"ms": round(wgrad_ms, 4), "TFLOP/s": round(flop / (wgrad_ms * 1e-3) / 1e12, 1),
+                          "frac_fp8_peak": round(flop / (wgrad_ms * 1e-3) / 1e12 / fp8_peak, 4),
+                          "dw_bytes": MOE_E * MOE_N * MOE_K * 4,
+                          "note": "dW_e [2048, 7168] fp32 for all 256 experts (15 GB written), "
+                                  "FLOPs counted over the real tokens; not part of the step"},
+        "ragged_128x1_quant": {"ms": round(rq_ms, 4), "GB/s": round(rq_bytes / (rq_ms * 1e-3) / 1e9, 1),
+                               "note": "dY and X of the expert rows to the grouped-Wgrad operand form"},
         "e2e": None,
         "e2e_note": "not measured for this secondary workload (the expert weights alone are 7.5 GB of H2D per step)",
         "gpu_launches": len(launches) * args.steps,

@@ -207,7 +207,7 @@ template <int MODE, int BN, bool GROUPED>
 int launch_gemm(const uint8_t* A, const float* sA, const uint8_t* B, const float* sB, void* D,
                 const int32_t* offsets, int E, int64_t M, int64_t N, int64_t K, cudaStream_t st,
                 void* workspace = nullptr, size_t ws_bytes = 0, bool accumulate = false,
-                uint8_t* q_out = nullptr, float* s_out = nullptr)
+                uint8_t* q_out = nullptr, float* s_out = nullptr, int64_t rows_total = -1)
 {
     using S = GemmShape<MODE, BN, GROUPED>;
     const int prep = prepare_kernel<MODE, BN, GROUPED>();
@@ -218,13 +218,16 @@ int launch_gemm(const uint8_t* A, const float* sA, const uint8_t* B, const float
         const uint64_t krows = GROUPED ? (uint64_t)E * (uint64_t)K : (uint64_t)K;
         if (!make_tmap_u8(&tb, B, (uint64_t)N, krows, 128, 128)) return FP8Q_ERR_CUDA;
     } else {
-        const uint64_t rows = GROUPED ? (uint64_t)E * (uint64_t)N : (uint64_t)N;
+        const uint64_t rows = (GROUPED && MODE != kModeWgrad) ? (uint64_t)E * (uint64_t)N : (uint64_t)N;
         if (!make_tmap_u8(&tb, B, (uint64_t)K, rows, 128, BN)) return FP8Q_ERR_CUDA;
     }
     CUtensorMap td, tq;   // the epilogue's store maps (the grouped GEMM stores without them)
     memset(&td, 0, sizeof(td));
     memset(&tq, 0, sizeof(tq));
-    if (!GROUPED && D && !make_tmap_out(&td, D, (uint64_t)N, (uint64_t)M, MODE == kModeWgrad ? 4 : 2))
+    // Row-grouped GEMMs store without a map; the K-grouped Wgrad stores expert e's dW at rows e*M.
+    const uint64_t d_rows = (GROUPED && MODE == kModeWgrad) ? (uint64_t)E * (uint64_t)M : (uint64_t)M;
+    if ((!GROUPED || MODE == kModeWgrad) && D &&
+        !make_tmap_out(&td, D, (uint64_t)N, d_rows, MODE == kModeWgrad ? 4 : 2))
         return FP8Q_ERR_CUDA;
     if (q_out && !make_tmap_out(&tq, q_out, (uint64_t)N, (uint64_t)M, 1)) return FP8Q_ERR_CUDA;
     GemmArgs a;
@@ -244,10 +247,13 @@ int launch_gemm(const uint8_t* A, const float* sA, const uint8_t* B, const float
     a.s_out = s_out;
     a.quant_out = q_out ? 1 : 0;
     a.store_d = D ? 1 : 0;
+    a.rows_total = rows_total >= 0 ? rows_total : M;
     const int sms = sm_count();
     if (sms <= 0) return FP8Q_ERR_CUDA;
-    // Grouped: at most ceil(Mtot/128) + E row tiles (each group adds at most one partial tile).
-    const int64_t m_tiles = GROUPED ? (M + 127) / 128 + E : (M + 127) / 128;
+    // Row-grouped: at most ceil(Mtot/128) + E row tiles (each group adds at most one partial
+    // tile).  K-grouped: E x the dense tiles.
+    const int64_t m_tiles = (GROUPED && MODE != kModeWgrad) ? (M + 127) / 128 + E
+                            : (GROUPED ? (int64_t)E * ((M + 127) / 128) : (M + 127) / 128);
     const int64_t tiles = m_tiles * (N / BN);
     const int64_t units = tiles * a.KB;
     if (!GROUPED && workspace && want_streamk(tiles, sms, a.KB)) {
@@ -556,6 +562,51 @@ int fp8_grouped_gemm_blockscaled_dgrad(const uint8_t* A, const float* sA, const 
     if (choose_bn(Mtot, N, E) == 256)
         return launch_gemm<kModeDgrad, 256, true>(A, sA, B, sB, D, offsets, E, Mtot, N, K, st);
     return launch_gemm<kModeDgrad, 128, true>(A, sA, B, sB, D, offsets, E, Mtot, N, K, st);
+}
+
+int fp8q_act_128x1_transposed_ragged(const uint16_t* x, const int32_t* offsets, int32_t E, int64_t Mtot, int64_t C,
+                                     uint8_t* qt, float* s, int64_t Kcap, fp8q_stream_t stream)
+{
+    if (E < 1 || Mtot < 0 || C < 0 || Kcap < 0) return FP8Q_ERR_ARG;
+    if (E > kRgMaxGroups) return FP8Q_ERR_UNSUPPORTED;
+    if (C % 64 != 0 || Kcap % 128 != 0) return FP8Q_ERR_SHAPE;
+    if (Mtot == 0 || C == 0) return FP8Q_OK;
+    if (!x || !offsets || !qt || !s) return FP8Q_ERR_ARG;
+    if (!aligned16(x) || !aligned16(qt) || !aligned16(s)) return FP8Q_ERR_ALIGN;
+    if ((reinterpret_cast<uintptr_t>(offsets) & 3u) != 0) return FP8Q_ERR_ALIGN;
+    const int64_t groups = (Mtot + 127) / 128 + E;   // padded token groups, at most
+    if (groups > 0x7FFFFFFF || Mtot >= (1ll << 31)) return FP8Q_ERR_UNSUPPORTED;
+    const int64_t chunks = (C / 64 + kRgChunk - 1) / kRgChunk;
+    const dim3 grid((unsigned)chunks, (unsigned)(groups < 65535 ? groups : 65535));
+    if (groups > 65535) return FP8Q_ERR_UNSUPPORTED;
+    return launch_kernel(act_128x1_t_ragged_kernel, grid, dim3(256), 0, (cudaStream_t)stream, false, x, offsets,
+                         (int)E, Mtot, C, qt, s, Kcap);
+}
+
+int fp8_grouped_gemm_blockscaled_wgrad(const uint8_t* A, const float* sA, const uint8_t* B, const float* sB,
+                                       const int32_t* offsets, int32_t E, int64_t Mtot, int64_t M, int64_t N,
+                                       int64_t Kcap, float* D, fp8q_stream_t stream)
+{
+    if (E < 1 || Mtot < 0 || M < 0 || N < 0 || Kcap < 0) return FP8Q_ERR_ARG;
+    if (E > 1024) return FP8Q_ERR_UNSUPPORTED;
+    if (M % 128 != 0 || N % 128 != 0 || Kcap % 128 != 0) return FP8Q_ERR_SHAPE;
+    if (M == 0 || N == 0) return FP8Q_OK;
+    if (Mtot >= (1ll << 31) || (int64_t)E * M >= (1ll << 31) || N >= (1ll << 31) || Kcap >= (1ll << 31))
+        return FP8Q_ERR_UNSUPPORTED;
+    if ((int64_t)E * (M / 128) * (N / 128) > 0x7FFFFFFF) return FP8Q_ERR_UNSUPPORTED;
+    if (!A || !sA || !B || !sB || !D || !offsets) return FP8Q_ERR_ARG;
+    if (!aligned16(A) || !aligned16(sA) || !aligned16(B) || !aligned16(sB) || !aligned16(D)) return FP8Q_ERR_ALIGN;
+    if ((reinterpret_cast<uintptr_t>(offsets) & 3u) != 0) return FP8Q_ERR_ALIGN;
+    const cudaStream_t st = (cudaStream_t)stream;
+    if (Kcap == 0) {
+        return cudaMemsetAsync(D, 0, (size_t)E * (size_t)M * (size_t)N * 4u, st) == cudaSuccess ? FP8Q_OK
+                                                                                             : FP8Q_ERR_CUDA;
+    }
+    if (choose_bn(M, N, E) == 256)
+        return launch_gemm<kModeWgrad, 256, true>(A, sA, B, sB, D, offsets, E, M, N, Kcap, st, nullptr, 0, false,
+                                                 nullptr, nullptr, Mtot);
+    return launch_gemm<kModeWgrad, 128, true>(A, sA, B, sB, D, offsets, E, M, N, Kcap, st, nullptr, 0, false,
+                                             nullptr, nullptr, Mtot);
 }
 
 int fp8q_selftest_wait_timeout(uint64_t limit_ns, fp8q_stream_t stream)

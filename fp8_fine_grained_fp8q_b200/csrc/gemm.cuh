@@ -56,6 +56,7 @@ struct GemmArgs {
     float* s_out;
     int32_t quant_out;
     int32_t store_d;
+    int64_t rows_total;       // grouped: the offsets must end here (rows of A, or tokens for Wgrad)
 };
 
 // One piece of work: groups [kb0, kb1) of tile `tile`.
@@ -149,19 +150,34 @@ struct GemmShape {
 };
 
 struct TileInfo {
-    int32_t row0;      // first row of the 128-row tile
+    int32_t row0;      // first row of the 128-row tile (rows of A)
     int32_t row_end;   // rows >= row_end are not part of this tile's group (masked)
     int32_t n0;        // first column
     int32_t e;         // group
+    int32_t out_row0;  // first row of the tile in D (K-grouped Wgrad: expert e's dW starts at e*M)
 };
 
-template <bool GROUPED>
+// Grouped GEMMs.  Row-grouped (Fprop / Dgrad): the rows of A are split among experts and a
+// tile holds one expert's rows.  K-grouped (Wgrad): every expert has the full M x N output, and
+// its K range is its own tokens' 128-token groups [g_pre[e], g_pre[e+1]).
+template <bool GROUPED, bool KGROUPED>
 __device__ __forceinline__ TileInfo decode_tile(int t, int nb_tiles, int bn, const GemmArgs& a,
                                                 const int32_t* g_off, const int32_t* g_pre)
 {
+    TileInfo ti;
+    if (KGROUPED) {
+        const int per_e = ((a.M + 127) >> 7) * nb_tiles;
+        ti.e = t / per_e;
+        const int r = t - ti.e * per_e;
+        const int mt = r / nb_tiles;
+        ti.n0 = (r - mt * nb_tiles) * bn;
+        ti.row0 = mt * 128;
+        ti.row_end = a.M;
+        ti.out_row0 = ti.e * a.M + ti.row0;
+        return ti;
+    }
     const int mt = t / nb_tiles;
     const int nt = t - mt * nb_tiles;
-    TileInfo ti;
     ti.n0 = nt * bn;
     if (GROUPED) {
         int lo = 0, hi = a.E;   // g_pre[lo] <= mt < g_pre[hi]
@@ -177,6 +193,7 @@ __device__ __forceinline__ TileInfo decode_tile(int t, int nb_tiles, int bn, con
         ti.row0 = mt * 128;
         ti.row_end = a.M;
     }
+    ti.out_row0 = ti.row0;
     return ti;
 }
 
@@ -273,7 +290,9 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
             run += cnt > 0 ? (cnt + 127) >> 7 : 0;
         }
         if (lane == 31) g_pre[E] = incl;
-        if (lane == 0) bad |= (g_off[0] != 0) || (g_off[E] != args.M);
+        if (lane == 0) bad |= (g_off[0] != 0) || ((int64_t)g_off[E] != args.rows_total);
+        // K-grouped: the experts' padded token groups must fit the operands' K extent.
+        if (MODE == kModeWgrad) bad |= __shfl_sync(0xFFFFFFFFu, incl, 31) > args.KB;
         bad = __any_sync(0xFFFFFFFFu, bad);
         if (bad && lane == 0) {
             misc[2] = 1;
@@ -286,8 +305,18 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
 
     const uint32_t tmem_base = misc[0];
     const int nb_tiles = args.N / BN;
-    const int num_m_tiles = GROUPED ? (misc[2] ? 0 : g_pre[args.E]) : (args.M + 127) / 128;
-    const int num_tiles = num_m_tiles * nb_tiles;
+    constexpr bool kKGrouped = GROUPED && MODE == kModeWgrad;    // K ranges per expert
+    constexpr bool kRowGrouped = GROUPED && MODE != kModeWgrad;  // rows per expert
+    const int num_m_tiles = kRowGrouped ? (misc[2] ? 0 : g_pre[args.E]) : (args.M + 127) / 128;
+    const int num_tiles = (kKGrouped ? (misc[2] ? 0 : args.E) : 1) * num_m_tiles * nb_tiles;
+    // K-grouped: a work item's K groups are its expert's padded token groups.
+    const auto kgroup_range = [&](WorkItem& it) {
+        if (kKGrouped) {
+            const int e = it.tile / (num_m_tiles * nb_tiles);
+            it.kb0 = g_pre[e];
+            it.kb1 = g_pre[e + 1];
+        }
+    };
     const int KB = args.KB;
 
     if (warp < 4) {
@@ -301,8 +330,9 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
             WorkSched ws = sched_begin(args);
             WorkItem it;
             while (ok && sched_next(ws, num_tiles, KB, it)) {
-                const TileInfo ti = decode_tile<GROUPED>(it.tile, nb_tiles, BN, args, g_off, g_pre);
-                const int brow = GROUPED ? ti.e * args.N + ti.n0 : ti.n0;
+                kgroup_range(it);
+                const TileInfo ti = decode_tile<GROUPED, kKGrouped>(it.tile, nb_tiles, BN, args, g_off, g_pre);
+                const int brow = kRowGrouped ? ti.e * args.N + ti.n0 : ti.n0;
                 for (int kb = it.kb0; kb < it.kb1; ++kb) {
                     if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) { ok = false; break; }
                     const uint32_t sa = smem_u32(smem + stage * S::kStageBytes);
@@ -346,6 +376,7 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
             WorkSched ws = sched_begin(args);
             WorkItem it;
             while (ok && sched_next(ws, num_tiles, KB, it)) {
+                kgroup_range(it);
                 for (int kb = it.kb0; kb < it.kb1; ++kb) {
                     if (tb == mybuf) {
                         if (!mbar_wait(tempty_bar(tb), tph ^ 1u, abort_flag)) { ok = false; break; }
@@ -414,7 +445,8 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
         WorkItem it;
         bool alive = true;
         while (alive && sched_next(wsched, num_tiles, KB, it)) {
-            const TileInfo ti = decode_tile<GROUPED>(it.tile, nb_tiles, BN, args, g_off, g_pre);
+            kgroup_range(it);
+            const TileInfo ti = decode_tile<GROUPED, kKGrouped>(it.tile, nb_tiles, BN, args, g_off, g_pre);
             const int row = ti.row0 + rit;
             const bool in_a = row < args.M;
             const int ncol0 = ti.n0 + half * S::kCols;
@@ -584,7 +616,7 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                 constexpr int kElt = (MODE == kModeWgrad) ? 4 : 2;    // bytes per output element
                 constexpr int kSlabCols = 64 / kElt;
                 uint4* stage0 = reinterpret_cast<uint4*>(smem + S::kOffEpi) + pw * 128 * S::kEpiBufs;
-                const int wrow0 = ti.row0 + quad * 32;
+                const int wrow0 = ti.out_row0 + quad * 32;
                 // Fused 1x128 quantisation: this thread's kCols = 128 columns of its row are one
                 // group.  Its scale comes from the bf16-rounded outputs, as the activation
                 // quantiser would see them in D.
@@ -620,7 +652,7 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                                               pack_bf16x2(acc[q + 3].x, acc[q + 3].y));
                         }
                     }
-                    if (!GROUPED) {
+                    if (!kRowGrouped) {
                         // The buffer is free once the store issued from it kEpiBufs slabs ago has
                         // read it.
                         if (lane == 0) bulk_wait_group_read<S::kEpiBufs - 1>();
@@ -644,7 +676,7 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
 #pragma unroll
                         for (int p = 0; p < 4; ++p) stage[lane * 4 + (p ^ wsw)] = u[p];
                     }
-                    if (!GROUPED) {
+                    if (!kRowGrouped) {
                         fence_proxy_async_smem();     // the writes above, before the async-proxy read
                         __syncwarp();
                         if (lane == 0) {
@@ -707,7 +739,7 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
         }
         // Every store has finished reading shared memory and writing its tile before the CTA
         // (and its shared memory) goes away.
-        if (!GROUPED && lane == 0) bulk_wait_group<0>();
+        if (!kRowGrouped && lane == 0) bulk_wait_group<0>();
         __syncwarp();
         tc_fence_before();
         named_bar_arrive(1, 32 + S::kPromoThreads);

@@ -186,6 +186,121 @@ __global__ void __launch_bounds__(256) act_128x1_t_kernel(const uint16_t* __rest
 }
 
 // ------------------------------------------------------------------------------------------
+// 128x1 with transposed output over expert-grouped rows (the grouped Wgrad operands).  Rows
+// offsets[e] .. offsets[e+1]-1 of x[Mtot, C] are expert e's tokens.  Expert e's 128-token groups
+// start at its first row; a final partial group takes its max-abs over the tokens it has.  In
+// the transposed output qt[C, Kcap] the expert's tokens start at column 128 * P[e],
+// P[e] = sum over e' < e of ceil(n_e' / 128), and the rest of its last group holds zero codes;
+// st[Kcap/128][C].  CTA (x, y): padded group g = y, channel blocks 8x .. 8x+7 of 64 channels.
+// Each CTA rebuilds P from the offsets (validated: 0-based, nondecreasing, ending at Mtot, and
+// P[E] <= Kcap/128; otherwise FP8Q_DEV_BAD_OFFSETS is latched and nothing is written).
+// ------------------------------------------------------------------------------------------
+constexpr int kRgMaxGroups = 1024;
+constexpr int kRgChunk = 8;   // 64-channel blocks per CTA
+
+__global__ void __launch_bounds__(256) act_128x1_t_ragged_kernel(const uint16_t* __restrict__ x,
+                                                                 const int32_t* __restrict__ offsets, int E,
+                                                                 int64_t Mtot, int64_t C, uint8_t* __restrict__ qt,
+                                                                 float* __restrict__ s, int64_t Kcap)
+{
+    griddep_launch_dependents();
+    griddep_wait();
+    __shared__ int s_off[kRgMaxGroups + 1];
+    __shared__ int s_pre[kRgMaxGroups + 1];
+    __shared__ float red[8][kT1Ch];
+    __shared__ float inv_c[kT1Ch];
+    __shared__ int s_bad;
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (w == 0) {
+        for (int i = lane; i <= E; i += 32) s_off[i] = __ldg(offsets + i);
+        __syncwarp();
+        const int per = (E + 31) >> 5;
+        const int lo = min(E, lane * per), hi = min(E, lo + per);
+        int local = 0;
+        bool bad = false;
+        for (int e = lo; e < hi; ++e) {
+            const int cnt = s_off[e + 1] - s_off[e];
+            bad |= cnt < 0;
+            local += cnt > 0 ? (cnt + 127) >> 7 : 0;
+        }
+        int incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        int run = incl - local;
+        for (int e = lo; e < hi; ++e) {
+            s_pre[e] = run;
+            const int cnt = s_off[e + 1] - s_off[e];
+            run += cnt > 0 ? (cnt + 127) >> 7 : 0;
+        }
+        if (lane == 31) s_pre[E] = incl;
+        const int total = __shfl_sync(0xFFFFFFFFu, incl, 31);   // padded groups of all experts
+        if (lane == 0) bad |= (s_off[0] != 0) || ((int64_t)s_off[E] != Mtot) || ((int64_t)total * 128 > Kcap);
+        bad = __any_sync(0xFFFFFFFFu, bad);
+        if (lane == 0) s_bad = bad ? 1 : 0;
+    }
+    __syncthreads();
+    if (s_bad) {
+        if (threadIdx.x == 0) latch_status(2 /* FP8Q_DEV_BAD_OFFSETS */);
+        return;
+    }
+    const int g = blockIdx.y;
+    if (g >= s_pre[E]) return;
+    int lo = 0, hi = E;   // s_pre[lo] <= g < s_pre[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (s_pre[mid] <= g) lo = mid; else hi = mid;
+    }
+    const int64_t r0 = (int64_t)s_off[lo] + 128ll * (g - s_pre[lo]);
+    const int nvalid = (int)min((int64_t)128, (int64_t)s_off[lo + 1] - r0);
+
+    for (int j = 0; j < kRgChunk; ++j) {
+        const int64_t c0 = ((int64_t)blockIdx.x * kRgChunk + j) * kT1Ch;
+        if (c0 >= C) break;
+        // Tokens 16w + i of the group, channels c0 + 2*lane and + 1; tokens past the expert's
+        // end read as zero.
+        const uint32_t* src = reinterpret_cast<const uint32_t*>(x + (r0 + 16 * w) * C + c0) + lane;
+        uint32_t v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = (16 * w + i < nvalid) ? __ldg(src + (size_t)i * (size_t)(C >> 1)) : 0u;
+        float m0 = 0.0f, m1 = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            m0 = fmaxf(m0, fabsf(bf16_lo(v[i])));
+            m1 = fmaxf(m1, fabsf(bf16_hi(v[i])));
+        }
+        red[w][2 * lane] = m0;
+        red[w][2 * lane + 1] = m1;
+        __syncthreads();
+        if (threadIdx.x < kT1Ch) {
+            float a = red[0][threadIdx.x];
+#pragma unroll
+            for (int k = 1; k < 8; ++k) a = fmaxf(a, red[k][threadIdx.x]);
+            float sc, inv;
+            group_scale(a, sc, inv);
+            s[(int64_t)g * C + c0 + threadIdx.x] = sc;
+            inv_c[threadIdx.x] = inv;
+        }
+        __syncthreads();
+        const float inv0 = inv_c[2 * lane], inv1 = inv_c[2 * lane + 1];
+        uint32_t q0[4], q1[4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            q0[p] = e4m3x2(__fmul_rn(bf16_lo(v[4 * p + 0]), inv0), __fmul_rn(bf16_lo(v[4 * p + 1]), inv0)) |
+                    (e4m3x2(__fmul_rn(bf16_lo(v[4 * p + 2]), inv0), __fmul_rn(bf16_lo(v[4 * p + 3]), inv0)) << 16);
+            q1[p] = e4m3x2(__fmul_rn(bf16_hi(v[4 * p + 0]), inv1), __fmul_rn(bf16_hi(v[4 * p + 1]), inv1)) |
+                    (e4m3x2(__fmul_rn(bf16_hi(v[4 * p + 2]), inv1), __fmul_rn(bf16_hi(v[4 * p + 3]), inv1)) << 16);
+        }
+        uint8_t* dst = qt + (c0 + 2 * lane) * Kcap + (int64_t)g * 128 + 16 * w;
+        *reinterpret_cast<uint4*>(dst) = make_uint4(q0[0], q0[1], q0[2], q0[3]);
+        *reinterpret_cast<uint4*>(dst + Kcap) = make_uint4(q1[0], q1[1], q1[2], q1[3]);
+        __syncthreads();   // red and inv_c are rewritten by the next channel block
+    }
+}
+
+// ------------------------------------------------------------------------------------------
 // Both activation forms in one pass: x[T,C] -> (q[T,C], s[C/128][T]) as the 1x128 kernel and
 // (qt[C,T], st[T/128][C]) as the 128x1 kernel, reading x once.  One CTA per 128-token x
 // 128-channel tile, which is a whole group in both directions.  Warp w holds tokens

@@ -53,6 +53,8 @@ def lib() -> ctypes.CDLL:
         "fp8_gemm_blockscaled_quant": [I, P, P, P, P, P, P, P, I64, I64, I64, P, ctypes.c_size_t, P],
         "fp8_grouped_gemm_blockscaled": [P, P, P, P, P, I32, I64, I64, I64, P, P],
         "fp8_grouped_gemm_blockscaled_dgrad": [P, P, P, P, P, I32, I64, I64, I64, P, P],
+        "fp8_grouped_gemm_blockscaled_wgrad": [P, P, P, P, P, I32, I64, I64, I64, I64, P, P],
+        "fp8q_act_128x1_transposed_ragged": [P, P, I32, I64, I64, P, P, I64, P],
         "fp8q_device_status": [P, ctypes.POINTER(I)],
     }.items():
         fn = getattr(L, name)
@@ -310,6 +312,51 @@ def grouped_gemm_blockscaled_dgrad(A: torch.Tensor, sA: torch.Tensor, B: torch.T
     _check("fp8_grouped_gemm_blockscaled_dgrad",
            lib().fp8_grouped_gemm_blockscaled_dgrad(_p(A), _p(sA), _p(B), _p(sB), _p(offsets), E, Mtot,
                                                     N, K, _p(out), _stream(A.device)))
+    return out
+
+
+def ragged_capacity(Mtot: int, E: int) -> int:
+    """A padded token extent that fits any routing of Mtot rows over E experts."""
+    return 128 * ((Mtot + 127) // 128 + E)
+
+
+def act_128x1_transposed_ragged(x: torch.Tensor, offsets: torch.Tensor, Kcap: int | None = None,
+                                qt: torch.Tensor | None = None, s: torch.Tensor | None = None):
+    """x[Mtot,C] bf16 rows grouped by expert (offsets int32[E+1] on the device) ->
+    (qt[C,Kcap] uint8, s[Kcap/128, C] fp32), each expert's 128-token groups padded to whole groups."""
+    _require(x, "x", torch.bfloat16, 2)
+    _require(offsets, "offsets", torch.int32, 1)
+    Mtot, C = x.shape
+    E = offsets.numel() - 1
+    Kcap = ragged_capacity(Mtot, E) if Kcap is None else Kcap
+    qt = _out(qt, (C, Kcap), torch.uint8, x.device, "qt")
+    s = _out(s, (Kcap // 128, C), torch.float32, x.device, "s")
+    _check("fp8q_act_128x1_transposed_ragged",
+           lib().fp8q_act_128x1_transposed_ragged(_p(x), _p(offsets), E, Mtot, C, _p(qt), _p(s), Kcap,
+                                                  _stream(x.device)))
+    return qt, s
+
+
+def grouped_gemm_blockscaled_wgrad(A: torch.Tensor, sA: torch.Tensor, B: torch.Tensor,
+                                   sB: torch.Tensor, offsets: torch.Tensor, Mtot: int,
+                                   out: torch.Tensor | None = None):
+    """Grouped Wgrad: A = dY^T codes [M,Kcap], sA[Kcap/128,M], B = X^T codes [N,Kcap],
+    sB[Kcap/128,N] (both from act_128x1_transposed_ragged with the same offsets over Mtot
+    tokens).  Returns dW[E,M,N] fp32."""
+    _require(A, "A", torch.uint8, 2)
+    _require(B, "B", torch.uint8, 2)
+    _require(sA, "sA", torch.float32, 2)
+    _require(sB, "sB", torch.float32, 2)
+    _require(offsets, "offsets", torch.int32, 1)
+    M, Kcap = A.shape
+    N, Kb = B.shape
+    if Kb != Kcap:
+        raise ValueError("A and B must share the padded token extent")
+    E = offsets.numel() - 1
+    out = _out(out, (E, M, N), torch.float32, A.device, "out")
+    _check("fp8_grouped_gemm_blockscaled_wgrad",
+           lib().fp8_grouped_gemm_blockscaled_wgrad(_p(A), _p(sA), _p(B), _p(sB), _p(offsets), E, Mtot, M, N,
+                                                    Kcap, _p(out), _stream(A.device)))
     return out
 
 

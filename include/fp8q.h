@@ -248,6 +248,37 @@ FP8Q_API int fp8_grouped_gemm_blockscaled_dgrad(const uint8_t* A, const float* s
                                                 int64_t N, int64_t K, uint16_t* D, fp8q_stream_t stream);
 
 /*
+ * 128x1 transposed quantisation over expert-grouped rows: the operand form of the grouped Wgrad
+ * (the groups lie along the tokens, [REPOST] paragraph 4).  Rows offsets[e] .. offsets[e+1]-1 of
+ * x [Mtot, C] (bf16) are expert e's tokens.  Expert e's 128-token groups start at its first row;
+ * a final partial group takes its max-abs over the tokens it has (equivalently: the expert's rows
+ * zero-padded to a multiple of 128).  With P[e] = sum over e' < e of ceil(n_e' / 128):
+ *   qt : [C, Kcap] codes; expert e's tokens at columns 128 P[e] .., zero codes in its padding
+ *   s  : [Kcap / 128, C] fp32 scales; group P[e] + j is expert e's j-th group
+ * Columns and groups at or past 128 P[E] are not written.  offsets: DEVICE int32 [E + 1], checked
+ * on the device (0-based, nondecreasing, ending at Mtot, 128 P[E] <= Kcap; otherwise
+ * FP8Q_DEV_BAD_OFFSETS is latched and nothing is written).  Kcap = 128 (ceil(Mtot/128) + E) always
+ * suffices.  C % 64 == 0 and Kcap % 128 == 0 (FP8Q_ERR_SHAPE); E <= 1024.
+ */
+FP8Q_API int fp8q_act_128x1_transposed_ragged(const uint16_t* x, const int32_t* offsets, int32_t E, int64_t Mtot,
+                                              int64_t C, uint8_t* qt, float* s, int64_t Kcap,
+                                              fp8q_stream_t stream);
+
+/*
+ * Grouped Wgrad: dW_e = dY_e^T X_e for every expert, each summing over its own tokens ([REPOST]
+ * paragraphs 2-3: Wgrad in FP8, FP32 gradients).  The operands are the ragged 128x1 forms above:
+ *   A  : dY^T codes [M, Kcap],  sA : [Kcap/128, M]   (fp8q_act_128x1_transposed_ragged of dY)
+ *   B  : X^T codes [N, Kcap],   sB : [Kcap/128, N]   (the same of X)
+ *   offsets : the token offsets [E + 1] both were quantised with (DEVICE int32), Mtot tokens
+ *   D  : fp32 [E, M, N]; an expert without tokens gets dW_e = 0.
+ * M % 128 == 0, N % 128 == 0, Kcap % 128 == 0 (FP8Q_ERR_SHAPE); E <= 1024.  Malformed offsets
+ * (including 128 P[E] > Kcap) latch FP8Q_DEV_BAD_OFFSETS and write nothing.
+ */
+FP8Q_API int fp8_grouped_gemm_blockscaled_wgrad(const uint8_t* A, const float* sA, const uint8_t* B, const float* sB,
+                                                const int32_t* offsets, int32_t E, int64_t Mtot, int64_t M, int64_t N,
+                                                int64_t Kcap, float* D, fp8q_stream_t stream);
+
+/*
  * Synchronise `stream`, then read and clear the device status word of the current device.
  * *out receives FP8Q_DEV_OK or the first error latched since the last call.  Returns FP8Q_OK,
  * FP8Q_ERR_ARG (out == NULL) or FP8Q_ERR_CUDA.

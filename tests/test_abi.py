@@ -158,6 +158,24 @@ def test_grouped_dgrad_host_checks(L):
     assert g(P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE + 2), 4, 128, 128, 128, P(FAKE), s) == ERR_ALIGN
 
 
+def test_ragged_and_grouped_wgrad_host_checks(L):
+    s = None
+    q = L.fp8q_act_128x1_transposed_ragged
+    assert q(P(FAKE), P(FAKE), 0, 128, 64, P(FAKE), P(FAKE), 256, s) == ERR_ARG          # E < 1
+    assert q(P(FAKE), P(FAKE), 2000, 128, 64, P(FAKE), P(FAKE), 256, s) == ERR_UNSUPPORTED
+    assert q(P(FAKE), P(FAKE), 4, 128, 65, P(FAKE), P(FAKE), 256, s) == ERR_SHAPE
+    assert q(P(FAKE), P(FAKE), 4, 128, 64, P(FAKE), P(FAKE), 200, s) == ERR_SHAPE       # Kcap % 128
+    assert q(P(FAKE), P(FAKE), 4, 0, 64, P(FAKE), P(FAKE), 256, s) == OK
+    assert q(P(FAKE), P(FAKE + 2), 4, 128, 64, P(FAKE), P(FAKE), 256, s) == ERR_ALIGN
+    g = L.fp8_grouped_gemm_blockscaled_wgrad
+    a = (P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE))
+    assert g(*a, 0, 128, 128, 128, 256, P(FAKE), s) == ERR_ARG
+    assert g(*a, 4, 128, 100, 128, 256, P(FAKE), s) == ERR_SHAPE
+    assert g(*a, 4, 128, 128, 128, 100, P(FAKE), s) == ERR_SHAPE
+    assert g(*a, 4, 128, 0, 128, 256, P(FAKE), s) == OK
+    assert g(*a, 4, 128, 128, 128, 256, None, s) == ERR_ARG
+
+
 def test_selftest_and_status_arg_checks(L):
     assert L.fp8q_selftest_wait_timeout(0, None) == ERR_ARG
     assert L.fp8q_selftest_wait_timeout(3_000_000_000, None) == ERR_ARG
