@@ -23,6 +23,11 @@ What it computes, from the pages on the DeepSeek-V3 Technical Report (arXiv 2412
 Readings the pages leave open (OCP E4M3FN, round-to-nearest-even with saturation at 448,
 max-abs scaling with an amax floor of 2^-100) are stated in ``fp8q_oracle.c``.
 
+The quantisers also take ``scale_fmt="ue8m0"``: a power-of-two scale (the smallest power of two
+not below the binary32 quotient a / 448), a separate mode the pages do not describe.  It is the
+scale format the block-scaled tensor-core MMA accepts; the GEMM oracle needs no change for it,
+since its scales are ordinary binary32 values.
+
 The arithmetic lives in ``fp8q_oracle.c``; this module only marshals numpy arrays (and, for the
 expert-grouped Wgrad operands, pads each expert's rows before calling it).
 """
@@ -36,6 +41,7 @@ import numpy as np
 from . import build as _build
 
 FPROP, DGRAD, WGRAD = 0, 1, 2
+SCALE_FORMATS = {"fp32": 0, "ue8m0": 1}
 
 _lib = None
 
@@ -53,9 +59,9 @@ def _load():
         lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
         lib.oracle_e4m3_encode_array.argtypes = [P, I64, P]
         lib.oracle_e4m3_decode_array.argtypes = [P, I64, P]
-        lib.oracle_quant_1x128.argtypes = [P, I64, I64, P, P]
-        lib.oracle_quant_128x1_t.argtypes = [P, I64, I64, P, P]
-        lib.oracle_quant_128x128.argtypes = [P, I64, I64, P, P, P]
+        lib.oracle_quant_1x128_fmt.argtypes = [P, I64, I64, P, P, ctypes.c_int]
+        lib.oracle_quant_128x1_t_fmt.argtypes = [P, I64, I64, P, P, ctypes.c_int]
+        lib.oracle_quant_128x128_fmt.argtypes = [P, I64, I64, P, P, P, ctypes.c_int]
         lib.oracle_gemm.argtypes = [ctypes.c_int, P, P, P, P, I64, I64, I64, P, P, P, P]
         lib.oracle_gemm_entries.argtypes = [ctypes.c_int, P, P, P, P, I64, I64, I64, P, P,
                                             I64, P, P]
@@ -107,35 +113,45 @@ def e4m3_decode(c) -> np.ndarray:
 # Quantisers
 # ----------------------------------------------------------------------------------------- #
 
-def quant_1x128(x_bits: np.ndarray):
+def _fmt(scale_fmt: str) -> int:
+    """"fp32": the pages' max-abs scale a / 448.  "ue8m0": its power-of-two variant, the
+    smallest power of two not below the binary32 quotient a / 448 (a separate mode the pages do
+    not describe: the scale format of the block-scaled tensor-core MMA)."""
+    try:
+        return SCALE_FORMATS[scale_fmt]
+    except KeyError:
+        raise ValueError(f"scale_fmt must be one of {sorted(SCALE_FORMATS)}") from None
+
+
+def quant_1x128(x_bits: np.ndarray, scale_fmt: str = "fp32"):
     """x[M,K] bf16 bits -> (q[M,K] uint8, s[K/128, M] float32)."""
     x = _bf16_bits(x_bits)
     M, K = x.shape
     q = np.empty((M, K), dtype=np.uint8)
     s = np.empty((K // 128, M), dtype=np.float32)
-    _load().oracle_quant_1x128(_ptr(x), M, K, _ptr(q), _ptr(s))
+    _load().oracle_quant_1x128_fmt(_ptr(x), M, K, _ptr(q), _ptr(s), _fmt(scale_fmt))
     return q, s
 
 
-def quant_128x1_t(x_bits: np.ndarray):
+def quant_128x1_t(x_bits: np.ndarray, scale_fmt: str = "fp32"):
     """x[T,C] bf16 bits -> (qt[C,T] uint8, s[T/128, C] float32)."""
     x = _bf16_bits(x_bits)
     T, C = x.shape
     qt = np.empty((C, T), dtype=np.uint8)
     s = np.empty((T // 128, C), dtype=np.float32)
-    _load().oracle_quant_128x1_t(_ptr(x), T, C, _ptr(qt), _ptr(s))
+    _load().oracle_quant_128x1_t_fmt(_ptr(x), T, C, _ptr(qt), _ptr(s), _fmt(scale_fmt))
     return qt, s
 
 
-def quant_128x128(w_bits: np.ndarray, want_transposed: bool = False):
+def quant_128x128(w_bits: np.ndarray, want_transposed: bool = False, scale_fmt: str = "fp32"):
     """w[N,K] bf16 bits -> (q[N,K], s[N/128, K/128], qt[K,N] or None)."""
     w = _bf16_bits(w_bits)
     N, K = w.shape
     q = np.empty((N, K), dtype=np.uint8)
     s = np.empty((N // 128, K // 128), dtype=np.float32)
     qt = np.empty((K, N), dtype=np.uint8) if want_transposed else None
-    _load().oracle_quant_128x128(_ptr(w), N, K, _ptr(q), _ptr(s),
-                                 _ptr(qt) if qt is not None else None)
+    _load().oracle_quant_128x128_fmt(_ptr(w), N, K, _ptr(q), _ptr(s),
+                                     _ptr(qt) if qt is not None else None, _fmt(scale_fmt))
     return q, s, qt
 
 
@@ -222,7 +238,7 @@ def ragged_group_prefix(offsets) -> np.ndarray:
     return P
 
 
-def quant_128x1_t_ragged(x_bits: np.ndarray, offsets):
+def quant_128x1_t_ragged(x_bits: np.ndarray, offsets, scale_fmt: str = "fp32"):
     """128x1 groups along each expert's own tokens, for the grouped Wgrad dW_e = dY_e^T X_e.
 
     x[Mtot, C] bf16 bits with rows ordered by expert (rows offsets[e] .. offsets[e+1]-1 are
@@ -245,7 +261,7 @@ def quant_128x1_t_ragged(x_bits: np.ndarray, offsets):
         g = int(P[e + 1] - P[e])
         block = np.zeros((128 * g, C), dtype=x_bits.dtype)
         block[:n] = x_bits[off[e]:off[e + 1]]
-        q, se = quant_128x1_t(block)
+        q, se = quant_128x1_t(block, scale_fmt=scale_fmt)
         qt[:, 128 * int(P[e]):128 * int(P[e + 1])] = q
         s[int(P[e]):int(P[e + 1])] = se
     return qt, s

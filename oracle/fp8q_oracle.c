@@ -28,6 +28,10 @@
  *     IEEE binary32 operations rounded to nearest.
  *   - The GEMM result is the exact dot product of the dequantised operands, accumulated here in
  *     binary64 (each dequantised value dec(q)*s is exact in binary64).
+ *   - Power-of-two (UE8M0) scale variant, a separate mode that the pages do not describe (it is
+ *     the scale format the block-scaled tensor-core MMA accepts): s is the smallest power of two
+ *     not below the binary32 quotient a / 448, and codes are E4M3(x * (1 / s)), where 1 / s is an
+ *     exact power of two.  The default mode is the one above.
  *
  * Build: gcc -O2 -std=c11 -fopenmp -ffp-contract=off -fno-fast-math -shared -fPIC.
  * No FMA contraction and no excess precision: every float operation below is one IEEE
@@ -136,17 +140,32 @@ static float bf16_to_float(uint16_t h)
 static const float AMAX_FLOOR = 0x1p-100f;
 static const float E4M3_MAX = 448.0f;
 
+/* Scale formats of the quantisers: the pages' max-abs scale, or its power-of-two variant. */
+enum { SCALE_FP32 = 0, SCALE_UE8M0 = 1 };
+
 /* Scale and inverse of one group from its largest magnitude. */
-static void group_scale(float amax, float* s, float* inv)
+static void group_scale(float amax, float* s, float* inv, int fmt)
 {
     const float a = amax > AMAX_FLOOR ? amax : AMAX_FLOOR;
+    if (fmt == SCALE_UE8M0) {
+        /* r = m * 2^e with m in [0.5, 1): the smallest power of two >= r is 2^(e-1) when r is
+         * itself a power of two (m = 0.5), else 2^e.  r >= 2^-109 and r < 2^120, so both
+         * 2^p and 2^-p are normal binary32 numbers. */
+        const float r = a / E4M3_MAX;
+        int e;
+        const float m = frexpf(r, &e);
+        const int p = (m == 0.5f) ? e - 1 : e;
+        *s = ldexpf(1.0f, p);
+        *inv = ldexpf(1.0f, -p);
+        return;
+    }
     *s = a / E4M3_MAX;        /* dequantisation multiplier, stored */
     *inv = E4M3_MAX / a;      /* quantisation multiplier */
 }
 
 /* 1x128 tile-wise quantisation of activations [SUMMARY, Key ideas, FP8 bullet]: one scale per row per
  * 128 consecutive columns.  x[M][K] bf16 bits -> q[M][K] codes, s[K/128][M] scales. */
-void oracle_quant_1x128(const uint16_t* x, int64_t M, int64_t K, uint8_t* q, float* s)
+void oracle_quant_1x128_fmt(const uint16_t* x, int64_t M, int64_t K, uint8_t* q, float* s, int fmt)
 {
     const int64_t KB = K / 128;
 #pragma omp parallel for schedule(static)
@@ -158,7 +177,7 @@ void oracle_quant_1x128(const uint16_t* x, int64_t M, int64_t K, uint8_t* q, flo
                 if (v > amax) amax = v;
             }
             float sc, inv;
-            group_scale(amax, &sc, &inv);
+            group_scale(amax, &sc, &inv, fmt);
             s[kb * M + m] = sc;
             for (int64_t k = kb * 128; k < kb * 128 + 128; ++k) {
                 const float scaled = bf16_to_float(x[m * K + k]) * inv;
@@ -171,7 +190,7 @@ void oracle_quant_1x128(const uint16_t* x, int64_t M, int64_t K, uint8_t* q, flo
 /* 128x1 quantisation along tokens with transposed output, the operand form Wgrad needs
  * because its inner dimension is the token dimension [REPOST, paragraph 4]:
  * x[T][C] bf16 bits -> qt[C][T] codes, s[T/128][C] scales (one per channel per 128 tokens). */
-void oracle_quant_128x1_t(const uint16_t* x, int64_t T, int64_t C, uint8_t* qt, float* s)
+void oracle_quant_128x1_t_fmt(const uint16_t* x, int64_t T, int64_t C, uint8_t* qt, float* s, int fmt)
 {
     const int64_t TB = T / 128;
 #pragma omp parallel for schedule(static)
@@ -183,7 +202,7 @@ void oracle_quant_128x1_t(const uint16_t* x, int64_t T, int64_t C, uint8_t* qt, 
                 if (v > amax) amax = v;
             }
             float sc, inv;
-            group_scale(amax, &sc, &inv);
+            group_scale(amax, &sc, &inv, fmt);
             s[tb * C + c] = sc;
             for (int64_t t = tb * 128; t < tb * 128 + 128; ++t) {
                 const float scaled = bf16_to_float(x[t * C + c]) * inv;
@@ -196,8 +215,8 @@ void oracle_quant_128x1_t(const uint16_t* x, int64_t T, int64_t C, uint8_t* qt, 
 /* 128x128 block-wise quantisation of weights [SUMMARY, Key ideas, FP8 bullet]: one scale per 128 output
  * rows x 128 input columns.  w[N][K] -> q[N][K], s[N/128][K/128]; qt[K][N] (optional, may be
  * NULL) receives the same codes transposed. */
-void oracle_quant_128x128(const uint16_t* w, int64_t N, int64_t K, uint8_t* q, float* s,
-                          uint8_t* qt)
+void oracle_quant_128x128_fmt(const uint16_t* w, int64_t N, int64_t K, uint8_t* q, float* s,
+                              uint8_t* qt, int fmt)
 {
     const int64_t NB = N / 128, KB = K / 128;
 #pragma omp parallel for collapse(2) schedule(static)
@@ -210,7 +229,7 @@ void oracle_quant_128x128(const uint16_t* w, int64_t N, int64_t K, uint8_t* q, f
                     if (v > amax) amax = v;
                 }
             float sc, inv;
-            group_scale(amax, &sc, &inv);
+            group_scale(amax, &sc, &inv, fmt);
             s[nb * KB + kb] = sc;
             for (int64_t n = nb * 128; n < nb * 128 + 128; ++n)
                 for (int64_t k = kb * 128; k < kb * 128 + 128; ++k) {
@@ -220,6 +239,22 @@ void oracle_quant_128x128(const uint16_t* w, int64_t N, int64_t K, uint8_t* q, f
                 }
         }
     }
+}
+
+/* The pages' scale format (fmt = SCALE_FP32). */
+void oracle_quant_1x128(const uint16_t* x, int64_t M, int64_t K, uint8_t* q, float* s)
+{
+    oracle_quant_1x128_fmt(x, M, K, q, s, SCALE_FP32);
+}
+
+void oracle_quant_128x1_t(const uint16_t* x, int64_t T, int64_t C, uint8_t* qt, float* s)
+{
+    oracle_quant_128x1_t_fmt(x, T, C, qt, s, SCALE_FP32);
+}
+
+void oracle_quant_128x128(const uint16_t* w, int64_t N, int64_t K, uint8_t* q, float* s, uint8_t* qt)
+{
+    oracle_quant_128x128_fmt(w, N, K, q, s, qt, SCALE_FP32);
 }
 
 /* ------------------------------------------------------------------------------------------ */
