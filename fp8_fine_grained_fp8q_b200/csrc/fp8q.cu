@@ -23,6 +23,8 @@ using namespace fp8q;
 constexpr int kMaxDevices = 64;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool valid_fmt(int f) { return f == FP8Q_SCALE_FP32 || f == FP8Q_SCALE_UE8M0; }
+bool pow2(int f) { return f == FP8Q_SCALE_UE8M0; }
 
 int sm_count()
 {
@@ -150,15 +152,15 @@ bool make_tmap_out(CUtensorMap* tm, void* base, uint64_t inner, uint64_t outer, 
 // ------------------------------------------------------------------------------------------
 // GEMM launch
 // ------------------------------------------------------------------------------------------
-template <int MODE, int BN, bool GROUPED>
+template <int MODE, int BN, bool GROUPED, bool MX = false>
 int prepare_kernel()
 {
-    using S = GemmShape<MODE, BN, GROUPED>;
+    using S = GemmShape<MODE, BN, GROUPED, MX>;
     static int ready[kMaxDevices] = {0};   // 1 ok, -1 unusable
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FP8Q_ERR_CUDA;
     if (ready[dev] == 0) {
-        auto kern = gemm_blockscaled_kernel<MODE, BN, GROUPED>;
+        auto kern = gemm_blockscaled_kernel<MODE, BN, GROUPED, MX>;
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmemBytes) != cudaSuccess)
             return FP8Q_ERR_CUDA;
         cudaFuncAttributes attr;
@@ -203,14 +205,14 @@ bool want_streamk(int64_t tiles, int ctas, int kb)
     return tiles % ctas != 0;
 }
 
-template <int MODE, int BN, bool GROUPED>
+template <int MODE, int BN, bool GROUPED, bool MX = false>
 int launch_gemm(const uint8_t* A, const float* sA, const uint8_t* B, const float* sB, void* D,
                 const int32_t* offsets, int E, int64_t M, int64_t N, int64_t K, cudaStream_t st,
                 void* workspace = nullptr, size_t ws_bytes = 0, bool accumulate = false,
                 uint8_t* q_out = nullptr, float* s_out = nullptr, int64_t rows_total = -1)
 {
-    using S = GemmShape<MODE, BN, GROUPED>;
-    const int prep = prepare_kernel<MODE, BN, GROUPED>();
+    using S = GemmShape<MODE, BN, GROUPED, MX>;
+    const int prep = prepare_kernel<MODE, BN, GROUPED, MX>();
     if (prep != FP8Q_OK) return prep;
     CUtensorMap ta, tb;
     if (!make_tmap_u8(&ta, A, (uint64_t)K, (uint64_t)M, 128, 128)) return FP8Q_ERR_CUDA;
@@ -265,13 +267,13 @@ int launch_gemm(const uint8_t* A, const float* sA, const uint8_t* B, const float
             a.stamp = next_stamp();
             a.units = units;
             // CTAs wait on each other's partials: launch them co-resident (cooperative launch).
-            return launch_kernel(gemm_blockscaled_kernel<MODE, BN, GROUPED>, dim3((unsigned)grid),
+            return launch_kernel(gemm_blockscaled_kernel<MODE, BN, GROUPED, MX>, dim3((unsigned)grid),
                                  dim3(S::kThreads), S::kSmemBytes, st, true, ta, tb, td, tq, a);
         }
     }
     const int grid = (int)(tiles < sms ? tiles : sms);
     if (grid <= 0) return FP8Q_OK;
-    return launch_kernel(gemm_blockscaled_kernel<MODE, BN, GROUPED>, dim3((unsigned)grid), dim3(S::kThreads),
+    return launch_kernel(gemm_blockscaled_kernel<MODE, BN, GROUPED, MX>, dim3((unsigned)grid), dim3(S::kThreads),
                          S::kSmemBytes, st, false, ta, tb, td, tq, a);
 }
 
@@ -287,13 +289,13 @@ int choose_bn(int64_t M, int64_t N, int extra_m_tiles)
     return (N % 256 == 0) ? 256 : 128;
 }
 
-template <int MODE>
+template <int MODE, bool MX = false>
 int gemm_mode(const uint8_t* A, const float* sA, const uint8_t* B, const float* sB, void* D, int64_t M,
               int64_t N, int64_t K, cudaStream_t st, void* ws, size_t ws_bytes, bool accumulate = false)
 {
     if (choose_bn(M, N, 0) == 256)
-        return launch_gemm<MODE, 256, false>(A, sA, B, sB, D, nullptr, 1, M, N, K, st, ws, ws_bytes, accumulate);
-    return launch_gemm<MODE, 128, false>(A, sA, B, sB, D, nullptr, 1, M, N, K, st, ws, ws_bytes, accumulate);
+        return launch_gemm<MODE, 256, false, MX>(A, sA, B, sB, D, nullptr, 1, M, N, K, st, ws, ws_bytes, accumulate);
+    return launch_gemm<MODE, 128, false, MX>(A, sA, B, sB, D, nullptr, 1, M, N, K, st, ws, ws_bytes, accumulate);
 }
 
 // Waits on an mbarrier that nothing ever arrives on, so the bounded wait must expire, latch
@@ -367,9 +369,10 @@ const char* fp8q_status_string(int status)
 
 int fp8q_abi_version(void) { return 1; }
 
-int fp8q_act_1x128(const uint16_t* x, int64_t M, int64_t K, uint8_t* q, float* s, fp8q_stream_t stream)
+int fp8q_act_1x128_fmt(const uint16_t* x, int64_t M, int64_t K, uint8_t* q, float* s, int scale_fmt,
+                       fp8q_stream_t stream)
 {
-    if (M < 0 || K < 0) return FP8Q_ERR_ARG;
+    if (M < 0 || K < 0 || !valid_fmt(scale_fmt)) return FP8Q_ERR_ARG;
     if (K % 128 != 0) return FP8Q_ERR_SHAPE;
     if (M == 0 || K == 0) return FP8Q_OK;
     if (!x || !q || !s) return FP8Q_ERR_ARG;
@@ -382,27 +385,39 @@ int fp8q_act_1x128(const uint16_t* x, int64_t M, int64_t K, uint8_t* q, float* s
     const int64_t want = (ntiles + 32 * kUnr - 1) / (32 * kUnr);   // blocks of 32 eight-lane groups
     const int64_t cap = (int64_t)sms * 8;
     const int grid = (int)(want < cap ? want : cap);
-    return launch_kernel(act_1x128_kernel<kUnr>, dim3(grid), dim3(256), 0, (cudaStream_t)stream, false, x, q, s,
-                         (int)M, (int)K);
+    const auto kern = pow2(scale_fmt) ? act_1x128_kernel<kUnr, true> : act_1x128_kernel<kUnr, false>;
+    return launch_kernel(kern, dim3(grid), dim3(256), 0, (cudaStream_t)stream, false, x, q, s, (int)M, (int)K);
 }
 
-int fp8q_act_128x1_transposed(const uint16_t* x, int64_t T, int64_t C, uint8_t* qt, float* s,
-                              fp8q_stream_t stream)
+int fp8q_act_1x128(const uint16_t* x, int64_t M, int64_t K, uint8_t* q, float* s, fp8q_stream_t stream)
 {
-    if (T < 0 || C < 0) return FP8Q_ERR_ARG;
+    return fp8q_act_1x128_fmt(x, M, K, q, s, FP8Q_SCALE_FP32, stream);
+}
+
+int fp8q_act_128x1_transposed_fmt(const uint16_t* x, int64_t T, int64_t C, uint8_t* qt, float* s, int scale_fmt,
+                                  fp8q_stream_t stream)
+{
+    if (T < 0 || C < 0 || !valid_fmt(scale_fmt)) return FP8Q_ERR_ARG;
     if (T % 128 != 0 || C % 64 != 0) return FP8Q_ERR_SHAPE;
     if (T == 0 || C == 0) return FP8Q_OK;
     if (!x || !qt || !s) return FP8Q_ERR_ARG;
     if (!aligned16(x) || !aligned16(qt) || !aligned16(s)) return FP8Q_ERR_ALIGN;
     if (T / 128 > 65535 || C / 64 > 0x7FFFFFFF) return FP8Q_ERR_UNSUPPORTED;
     const dim3 grid((unsigned)(C / 64), (unsigned)(T / 128));
-    return launch_kernel(act_128x1_t_kernel, grid, dim3(256), 0, (cudaStream_t)stream, false, x, qt, s, T, C);
+    const auto kern = pow2(scale_fmt) ? act_128x1_t_kernel<true> : act_128x1_t_kernel<false>;
+    return launch_kernel(kern, grid, dim3(256), 0, (cudaStream_t)stream, false, x, qt, s, T, C);
 }
 
-int fp8q_act_dual(const uint16_t* x, int64_t T, int64_t C, uint8_t* q, float* s, uint8_t* qt, float* st,
-                  fp8q_stream_t stream)
+int fp8q_act_128x1_transposed(const uint16_t* x, int64_t T, int64_t C, uint8_t* qt, float* s,
+                              fp8q_stream_t stream)
 {
-    if (T < 0 || C < 0) return FP8Q_ERR_ARG;
+    return fp8q_act_128x1_transposed_fmt(x, T, C, qt, s, FP8Q_SCALE_FP32, stream);
+}
+
+int fp8q_act_dual_fmt(const uint16_t* x, int64_t T, int64_t C, uint8_t* q, float* s, uint8_t* qt, float* st,
+                      int scale_fmt, fp8q_stream_t stream)
+{
+    if (T < 0 || C < 0 || !valid_fmt(scale_fmt)) return FP8Q_ERR_ARG;
     if (T % 128 != 0 || C % 128 != 0) return FP8Q_ERR_SHAPE;
     if (T == 0 || C == 0) return FP8Q_OK;
     if (!x || !q || !s || !qt || !st) return FP8Q_ERR_ARG;
@@ -410,14 +425,21 @@ int fp8q_act_dual(const uint16_t* x, int64_t T, int64_t C, uint8_t* q, float* s,
         return FP8Q_ERR_ALIGN;
     if (T / 128 > 65535 || C / 128 > 0x7FFFFFFF) return FP8Q_ERR_UNSUPPORTED;
     const dim3 grid((unsigned)(C / 128), (unsigned)(T / 128));
-    return launch_kernel(act_dual_kernel, grid, dim3(256), 0, (cudaStream_t)stream, false, x, q, s, qt, st, T, C);
+    const auto kern = pow2(scale_fmt) ? act_dual_kernel<true> : act_dual_kernel<false>;
+    return launch_kernel(kern, grid, dim3(256), 0, (cudaStream_t)stream, false, x, q, s, qt, st, T, C);
 }
 
-int fp8q_quant_forward(const uint16_t* x, int64_t T, int64_t C, uint8_t* xq, float* xs, uint8_t* xqt, float* xst,
-                       const uint16_t* w, int64_t N, uint8_t* wq, float* ws, uint8_t* wqt_or_null,
-                       fp8q_stream_t stream)
+int fp8q_act_dual(const uint16_t* x, int64_t T, int64_t C, uint8_t* q, float* s, uint8_t* qt, float* st,
+                  fp8q_stream_t stream)
 {
-    if (T < 0 || C < 0 || N < 0) return FP8Q_ERR_ARG;
+    return fp8q_act_dual_fmt(x, T, C, q, s, qt, st, FP8Q_SCALE_FP32, stream);
+}
+
+int fp8q_quant_forward_fmt(const uint16_t* x, int64_t T, int64_t C, uint8_t* xq, float* xs, uint8_t* xqt,
+                           float* xst, const uint16_t* w, int64_t N, uint8_t* wq, float* ws, uint8_t* wqt_or_null,
+                           int scale_fmt, fp8q_stream_t stream)
+{
+    if (T < 0 || C < 0 || N < 0 || !valid_fmt(scale_fmt)) return FP8Q_ERR_ARG;
     if (T % 128 != 0 || C % 128 != 0 || N % 128 != 0) return FP8Q_ERR_SHAPE;
     if (C == 0 || (T == 0 && N == 0)) return FP8Q_OK;
     if (!x || !xq || !xs || !xqt || !xst || !w || !wq || !ws) return FP8Q_ERR_ARG;
@@ -426,22 +448,36 @@ int fp8q_quant_forward(const uint16_t* x, int64_t T, int64_t C, uint8_t* xq, flo
         return FP8Q_ERR_ALIGN;
     const int64_t tiles = (T / 128 + N / 128) * (C / 128);
     if (tiles > 0x7FFFFFFF) return FP8Q_ERR_UNSUPPORTED;
-    return launch_kernel(forward_operands_kernel, dim3((unsigned)tiles), dim3(256), 0, (cudaStream_t)stream, false, x,
-                         xq, xs, xqt, xst, T, C, w, wq, ws, wqt_or_null, N);
+    const auto kern = pow2(scale_fmt) ? forward_operands_kernel<true> : forward_operands_kernel<false>;
+    return launch_kernel(kern, dim3((unsigned)tiles), dim3(256), 0, (cudaStream_t)stream, false, x, xq, xs, xqt, xst,
+                         T, C, w, wq, ws, wqt_or_null, N);
 }
 
-int fp8q_weight_128x128(const uint16_t* w, int64_t N, int64_t K, uint8_t* q, float* s, uint8_t* qt_or_null,
-                        fp8q_stream_t stream)
+int fp8q_quant_forward(const uint16_t* x, int64_t T, int64_t C, uint8_t* xq, float* xs, uint8_t* xqt, float* xst,
+                       const uint16_t* w, int64_t N, uint8_t* wq, float* ws, uint8_t* wqt_or_null,
+                       fp8q_stream_t stream)
 {
-    if (N < 0 || K < 0) return FP8Q_ERR_ARG;
+    return fp8q_quant_forward_fmt(x, T, C, xq, xs, xqt, xst, w, N, wq, ws, wqt_or_null, FP8Q_SCALE_FP32, stream);
+}
+
+int fp8q_weight_128x128_fmt(const uint16_t* w, int64_t N, int64_t K, uint8_t* q, float* s, uint8_t* qt_or_null,
+                            int scale_fmt, fp8q_stream_t stream)
+{
+    if (N < 0 || K < 0 || !valid_fmt(scale_fmt)) return FP8Q_ERR_ARG;
     if (N % 128 != 0 || K % 128 != 0) return FP8Q_ERR_SHAPE;
     if (N == 0 || K == 0) return FP8Q_OK;
     if (!w || !q || !s) return FP8Q_ERR_ARG;
     if (!aligned16(w) || !aligned16(q) || !aligned16(s) || !aligned16(qt_or_null)) return FP8Q_ERR_ALIGN;
     if (N / 128 > 65535 || K / 128 > 0x7FFFFFFF) return FP8Q_ERR_UNSUPPORTED;
     const dim3 grid((unsigned)(K / 128), (unsigned)(N / 128));
-    return launch_kernel(weight_128x128_kernel, grid, dim3(256), 0, (cudaStream_t)stream, false, w, q, s, qt_or_null,
-                         N, K);
+    const auto kern = pow2(scale_fmt) ? weight_128x128_kernel<true> : weight_128x128_kernel<false>;
+    return launch_kernel(kern, grid, dim3(256), 0, (cudaStream_t)stream, false, w, q, s, qt_or_null, N, K);
+}
+
+int fp8q_weight_128x128(const uint16_t* w, int64_t N, int64_t K, uint8_t* q, float* s, uint8_t* qt_or_null,
+                        fp8q_stream_t stream)
+{
+    return fp8q_weight_128x128_fmt(w, N, K, q, s, qt_or_null, FP8Q_SCALE_FP32, stream);
 }
 
 size_t fp8q_gemm_workspace_size(int mode, int64_t M, int64_t N, int64_t K)
@@ -475,6 +511,31 @@ int fp8_gemm_blockscaled(int mode, const uint8_t* A, const float* sA, const uint
     case FP8Q_DGRAD: return gemm_mode<kModeDgrad>(A, sA, B, sB, D, M, N, K, st, workspace, ws_bytes);
     case FP8Q_WGRAD: return gemm_mode<kModeWgrad>(A, sA, B, sB, D, M, N, K, st, workspace, ws_bytes);
     default: return gemm_mode<kModeWgrad>(A, sA, B, sB, D, M, N, K, st, workspace, ws_bytes, true);
+    }
+}
+
+int fp8_gemm_blockscaled_ue8m0(int mode, const uint8_t* A, const float* sA, const uint8_t* B, const float* sB,
+                               void* D, int64_t M, int64_t N, int64_t K, void* workspace, size_t ws_bytes,
+                               fp8q_stream_t stream)
+{
+    if (mode != FP8Q_FPROP && mode != FP8Q_DGRAD && mode != FP8Q_WGRAD && mode != FP8Q_WGRAD_ACC) return FP8Q_ERR_ARG;
+    if (M < 0 || N < 0 || K < 0) return FP8Q_ERR_ARG;
+    if (N % 128 != 0 || K % 128 != 0) return FP8Q_ERR_SHAPE;
+    if (M == 0 || N == 0) return FP8Q_OK;
+    if (M >= (1ll << 31) || N >= (1ll << 31) || K >= (1ll << 31)) return FP8Q_ERR_UNSUPPORTED;
+    if (!A || !sA || !B || !sB || !D) return FP8Q_ERR_ARG;
+    if (!aligned16(A) || !aligned16(sA) || !aligned16(B) || !aligned16(sB) || !aligned16(D)) return FP8Q_ERR_ALIGN;
+    if (K == 0) {
+        if (mode == FP8Q_WGRAD_ACC) return FP8Q_OK;
+        const size_t bytes = (size_t)M * (size_t)N * (mode == FP8Q_WGRAD ? 4u : 2u);
+        return cudaMemsetAsync(D, 0, bytes, (cudaStream_t)stream) == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+    }
+    const cudaStream_t st = (cudaStream_t)stream;
+    switch (mode) {
+    case FP8Q_FPROP: return gemm_mode<kModeFprop, true>(A, sA, B, sB, D, M, N, K, st, workspace, ws_bytes);
+    case FP8Q_DGRAD: return gemm_mode<kModeDgrad, true>(A, sA, B, sB, D, M, N, K, st, workspace, ws_bytes);
+    case FP8Q_WGRAD: return gemm_mode<kModeWgrad, true>(A, sA, B, sB, D, M, N, K, st, workspace, ws_bytes);
+    default: return gemm_mode<kModeWgrad, true>(A, sA, B, sB, D, M, N, K, st, workspace, ws_bytes, true);
     }
 }
 
@@ -579,7 +640,7 @@ int fp8q_act_128x1_transposed_ragged(const uint16_t* x, const int32_t* offsets, 
     const int64_t chunks = (C / 64 + kRgChunk - 1) / kRgChunk;
     const dim3 grid((unsigned)chunks, (unsigned)(groups < 65535 ? groups : 65535));
     if (groups > 65535) return FP8Q_ERR_UNSUPPORTED;
-    return launch_kernel(act_128x1_t_ragged_kernel, grid, dim3(256), 0, (cudaStream_t)stream, false, x, offsets,
+    return launch_kernel(act_128x1_t_ragged_kernel<false>, grid, dim3(256), 0, (cudaStream_t)stream, false, x, offsets,
                          (int)E, Mtot, C, qt, s, Kcap);
 }
 

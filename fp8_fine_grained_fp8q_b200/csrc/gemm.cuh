@@ -107,7 +107,12 @@ __device__ __forceinline__ bool sched_next(WorkSched& w, int num_tiles, int KB, 
     return true;
 }
 
-template <int MODE, int BN, bool GROUPED>
+// MX: the power-of-two (UE8M0) scale variant.  The tensor core applies the scales itself
+// (tcgen05.mma kind::mxf8f6f4, one 8-bit exponent per row / column per 32-element K block), so
+// the whole K accumulates in one TMEM accumulator and the promotion warps only drain it once
+// per work item.  Warp 2 turns each K group's fp32 power-of-two scales into the scale-factor
+// layout the MMA reads and warp 1 copies them into TMEM (tcgen05.cp) ahead of the group's MMAs.
+template <int MODE, int BN, bool GROUPED, bool MX = false>
 struct GemmShape {
     static constexpr int kBM = 128;
     static constexpr int kBK = 128;
@@ -115,7 +120,16 @@ struct GemmShape {
     static constexpr int kBBytes = BN * kBK;
     static constexpr int kStageBytes = kABytes + kBBytes;
     static constexpr int kStages = (BN == 256) ? 4 : 6;
-    static constexpr int kScaleStages = (MODE == kModeWgrad) ? 4 : 0;
+    static constexpr int kScaleStages = (MODE == kModeWgrad && !MX) ? 4 : 0;
+    // MX scale factors per stage: one 512-byte chunk for A's 128 rows and one per 128 columns
+    // of B.  Chunk row r (16 bytes, r = 0..31) holds the exponents of rows r, 32 + r, 64 + r,
+    // 96 + r as four 32-bit words, each word the same exponent in all four bytes (one per
+    // 32-element K block of the 128-wide group); tcgen05.cp 32x128b.warpx4 copies a chunk to
+    // 4 TMEM columns of all 128 lanes, the layout the block-scaled MMA reads.
+    static constexpr int kSfChunks = MX ? 1 + BN / 128 : 0;
+    static constexpr int kSfStageBytes = 512 * kSfChunks;
+    static constexpr int kSfCol0 = BN;                   // TMEM: accumulator [0, BN), then 16 columns per stage
+    static constexpr int kOffSf = kStages * kStageBytes;
     // Promotion warpgroups.  Each owns BN / kPW columns of the tile (all 128 rows; warp w of a
     // group reads TMEM lanes 32*(w%4) ..).  Two: four groups (640 threads) halve each thread's
     // arithmetic per K group but not its TMEM round trips, which set the fold's length; with
@@ -127,26 +141,30 @@ struct GemmShape {
     static constexpr int kTmemCols = 2 * BN;       // two partial buffers
     static constexpr int kThreads = 128 + kPromoThreads;
     static constexpr int kMaxGroups = 1024;
-    static constexpr int kOffScales = kStages * kStageBytes;
+    static constexpr int kOffScales = kOffSf + kStages * kSfStageBytes;
     static constexpr int kOffBars = kOffScales + kScaleStages * BN * 4;
-    static constexpr int kNumBars = 2 * kStages + 4 + 2 * kScaleStages + 2;
+    static constexpr int kNumBars = 2 * kStages + 4 + 2 * kScaleStages + 2 + (MX ? kStages : 0);
     static constexpr int kOffMisc = kOffBars + kNumBars * 8;
     static constexpr int kOffGroups = kOffMisc + 16;
     // Epilogue staging: 2 KB per promotion warp and buffer, 1024-byte aligned (the 64-byte
     // swizzle of the tensor store works on absolute shared-memory address bits).  Two buffers per
     // warp where shared memory allows, so one slab's store reads while the next is written.
-    static constexpr int kEpiBufs = (MODE == kModeWgrad || GROUPED || kPW == 4) ? 1 : 2;
+    static constexpr int kEpiBufs = (MODE == kModeWgrad || GROUPED || kPW == 4 || MX) ? 1 : 2;
     static constexpr int kOffEpi = (kOffGroups + (GROUPED ? 2 * (kMaxGroups + 1) * 4 : 0) + 1023) / 1024 * 1024;
     static constexpr int kSmemBytes = kOffEpi + kPromoWarps * 2048 * kEpiBufs + 1024;
     // Registers (setmaxnreg moves them from the producer / MMA warpgroup to the promotion
     // warpgroups within the launch allocation):
     //   384 threads launched at 168:  128 x 40 + 256 x 232 = 64512 <= 384 x 168
     //   640 threads launched at  96:  128 x 56 + 512 x 104 = 60416 <= 640 x  96
-    static constexpr int kRegsLow = (kPW == 4) ? 56 : 40;
-    static constexpr int kRegsHigh = (kPW == 4) ? 104 : 232;
+    //   MX, 384 threads at 168:       128 x 72 + 256 x 216 = 64512 (the scale warp keeps two
+    //                                 K groups of scales in flight; the drain needs no scales)
+    static constexpr int kRegsLow = (kPW == 4) ? 56 : (MX ? 72 : 40);
+    static constexpr int kRegsHigh = (kPW == 4) ? 104 : (MX ? 216 : 232);
     static constexpr int kRegsLaunch = (kPW == 4) ? 96 : 168;
     static_assert(kThreads * kRegsLaunch >= 128 * kRegsLow + kPromoThreads * kRegsHigh, "register split");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+    static_assert(!MX || kSfCol0 + 16 * kStages <= kTmemCols, "MX scale factors fit the TMEM allocation");
+    static_assert(!(MX && GROUPED), "the MX variant is dense only");
 };
 
 struct TileInfo {
@@ -203,13 +221,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
     return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-template <int MODE, int BN, bool GROUPED>
-__global__ void __launch_bounds__(GemmShape<MODE, BN, GROUPED>::kThreads, 1)
+template <int MODE, int BN, bool GROUPED, bool MX = false>
+__global__ void __launch_bounds__(GemmShape<MODE, BN, GROUPED, MX>::kThreads, 1)
 gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmD, const __grid_constant__ CUtensorMap tmQ,
                         const GemmArgs args)
 {
-    using S = GemmShape<MODE, BN, GROUPED>;
+    using S = GemmShape<MODE, BN, GROUPED, MX>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float* col_scales = reinterpret_cast<float*>(smem + S::kOffScales);
@@ -227,6 +245,7 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
     const auto sempty_bar = [&](int s) { return bar0 + 8u * (2 * S::kStages + 4 + S::kScaleStages + s); };
     const uint32_t drain_bar = bar0 + 8u * (2 * S::kStages + 4 + 2 * S::kScaleStages);
     const uint32_t parked_bar = drain_bar + 8u;   // stream-K: all promotion warps wrote the slot
+    const auto sf_full_bar = [&](int s) { return parked_bar + 8u * (1 + s); };   // MX: chunks of stage s built
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -246,8 +265,10 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
             mbar_init(sfull_bar(s), 1);
             mbar_init(sempty_bar(s), S::kPromoWarps);
         }
-        mbar_init(drain_bar, 2);
+        mbar_init(drain_bar, MX ? 1 : 2);
         mbar_init(parked_bar, S::kPromoWarps);
+        if (MX)
+            for (int s = 0; s < S::kStages; ++s) mbar_init(sf_full_bar(s), 1);
         misc[1] = 0;
         misc[2] = 0;
         fence_mbar_init();
@@ -347,7 +368,7 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                     } else {
                         tma_load_2d(sb, &tmB, kb * 128, brow, full_bar(stage));
                     }
-                    if (MODE == kModeWgrad) {
+                    if (MODE == kModeWgrad && !MX) {
                         if (!mbar_wait(sempty_bar(ss), sph ^ 1u, abort_flag)) { ok = false; break; }
                         mbar_arrive_expect_tx(sfull_bar(ss), BN * 4);
                         bulk_load(smem_u32(col_scales + ss * BN), args.sB + (size_t)kb * args.N + ti.n0, BN * 4,
@@ -363,7 +384,135 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                 while (globaltimer_ns() - t0 < 50000ull) __nanosleep(1000);
             }
         }
-        } else if (warp == 1 || warp == 3) {
+        } else if (MX && warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (MX)
+        // One accumulator: a work item's groups accumulate into TMEM columns [0, BN); the next
+        // item starts once the promotion warps have drained it.  Per group: the scale chunks go
+        // to this stage's 16 TMEM scale columns (A at +0, B at +4), then 4 MMAs.  The four bytes
+        // of a scale word are one group's exponent for its four 32-element K blocks, all equal,
+        // so every MMA reads byte 0 (scale-factor id 0).
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0, aph = 0;
+            bool ok = true;
+            WorkSched ws = sched_begin(args);
+            WorkItem it;
+            while (ok && sched_next(ws, num_tiles, KB, it)) {
+                if (!mbar_wait(tempty_bar(0), aph ^ 1u, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                for (int kb = it.kb0; kb < it.kb1; ++kb) {
+                    if (!mbar_wait(full_bar(stage), phase, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait(sf_full_bar(stage), phase, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(smem + stage * S::kStageBytes);
+                    const uint32_t sb = sa + S::kABytes;
+                    const uint32_t sf = smem_u32(smem + S::kOffSf + stage * S::kSfStageBytes);
+                    const uint32_t tsf = tmem_base + (uint32_t)(S::kSfCol0 + 16 * stage);
+#pragma unroll
+                    for (int c = 0; c < S::kSfChunks; ++c) tmem_cp_32x128b_x4(tsf + 4u * c, sdesc_plain(sf + 512u * c, 128));
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint64_t ad = sdesc_sw128(sa + k * 32, 16, 1024);
+                        const uint64_t bd = (MODE == kModeDgrad) ? sdesc_sw128(sb + k * 4096, 16384, 1024)
+                                                                 : sdesc_sw128(sb + k * 32, 16, 1024);
+                        constexpr uint32_t idesc = idesc_mx_e4m3(BN, MODE == kModeDgrad, 0u, 0u);
+                        mma_mxf8f6f4(tmem_base, ad, bd, idesc, tsf, tsf + 4u, (kb > it.kb0 || k > 0) ? 1u : 0u);
+                    }
+                    tc_commit(empty_bar(stage));
+                    if (++stage == S::kStages) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                tc_commit(tfull_bar(0));
+                aph ^= 1u;
+            }
+            tc_commit(drain_bar);
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(drain_bar, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+            }
+        }
+        __syncwarp();
+        // Release TMEM once the promotion warps have read their last accumulator.
+        named_bar_sync(1, 32 + S::kPromoThreads);
+        tc_fence_after();
+        tmem_dealloc(tmem_base, S::kTmemCols);
+        } else if (MX && warp == 2) {
+        // ------------------------------------------------------------ scale chunks (MX)
+        // Lane l builds chunk row l: the exponents of A rows l + 32j (j = 0..3) and of B columns
+        // 128h + l + 32j.  The fp32 scales are loaded two K groups ahead (they come from L2:
+        // the item's scales are prefetched at its start); a scale that is not a positive normal
+        // power of two latches FP8Q_DEV_BAD_SCALES.
+        constexpr int kNB = (MODE == kModeWgrad) ? 4 * (BN / 128) : (BN / 128);   // B scales per lane
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true, bad = false;
+        WorkSched ws = sched_begin(args);
+        WorkItem it;
+        while (ok && sched_next(ws, num_tiles, KB, it)) {
+            const TileInfo ti = decode_tile<false, false>(it.tile, nb_tiles, BN, args, g_off, g_pre);
+            const auto a_ptr = [&](int kb, int j) -> const float* {
+                return args.sA + (size_t)kb * args.M + (ti.row0 + lane + 32 * j);
+            };
+            const auto b_ptr = [&](int kb, int j) -> const float* {
+                if (MODE == kModeWgrad) return args.sB + (size_t)kb * args.N + ti.n0 + 128 * (j >> 2) + lane + 32 * (j & 3);
+                if (MODE == kModeFprop) return args.sB + (size_t)((ti.n0 >> 7) + j) * KB + kb;
+                return args.sB + (size_t)kb * (args.N >> 7) + (ti.n0 >> 7) + j;
+            };
+            // Pull the item's scales into L2: per group 4 lines of row scales (and for Wgrad 8 of
+            // column scales), clamped to rows that exist.
+            for (int k = it.kb0 + (lane >> 3); k < it.kb1; k += 4) {
+                const int j = lane & 7;
+                if (j < 4) prefetch_l2(args.sA + (size_t)k * args.M + min(ti.row0 + 32 * j, args.M - 1));
+                if (MODE == kModeWgrad) {
+                    if (32 * j < BN) prefetch_l2(args.sB + (size_t)k * args.N + ti.n0 + 32 * j);
+                }
+                else if (j == 4) prefetch_l2(b_ptr(k, 0));
+            }
+            float na[3][4], nbv[3][kNB];
+            const auto load = [&](int kb, float (&a)[4], float (&b)[kNB]) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) a[j] = (kb < it.kb1 && ti.row0 + lane + 32 * j < args.M) ? __ldg(a_ptr(kb, j)) : 1.0f;
+#pragma unroll
+                for (int j = 0; j < kNB; ++j) b[j] = kb < it.kb1 ? __ldg(b_ptr(kb, j)) : 1.0f;
+            };
+            load(it.kb0, na[0], nbv[0]);
+            load(it.kb0 + 1, na[1], nbv[1]);
+            for (int kb = it.kb0; kb < it.kb1; ++kb) {
+                load(kb + 2, na[2], nbv[2]);
+                const auto expo = [&](float v) -> uint32_t {
+                    const uint32_t u = __float_as_uint(v);
+                    const uint32_t e = u >> 23;
+                    bad |= (u & 0x7FFFFFu) != 0u || e == 0u || e >= 255u;
+                    return (e & 0xFFu) * 0x01010101u;
+                };
+                const uint4 wa = make_uint4(expo(na[0][0]), expo(na[0][1]), expo(na[0][2]), expo(na[0][3]));
+                uint4 wb[BN / 128];
+#pragma unroll
+                for (int h = 0; h < BN / 128; ++h) {
+                    if (MODE == kModeWgrad) {
+                        wb[h] = make_uint4(expo(nbv[0][4 * h]), expo(nbv[0][4 * h + 1]), expo(nbv[0][4 * h + 2]),
+                                           expo(nbv[0][4 * h + 3]));
+                    } else {
+                        const uint32_t w = expo(nbv[0][h]);
+                        wb[h] = make_uint4(w, w, w, w);
+                    }
+                }
+                if (!warp_wait(empty_bar(stage), phase ^ 1u, abort_flag)) { ok = false; break; }
+                uint4* chunk = reinterpret_cast<uint4*>(smem + S::kOffSf + stage * S::kSfStageBytes);
+                chunk[lane] = wa;
+#pragma unroll
+                for (int h = 0; h < BN / 128; ++h) chunk[32 * (1 + h) + lane] = wb[h];
+                fence_proxy_async_smem();   // generic-proxy writes, read by tcgen05.cp
+                __syncwarp();
+                if (lane == 0) mbar_arrive(sf_full_bar(stage));
+                if (++stage == S::kStages) { stage = 0; phase ^= 1u; }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) { na[0][j] = na[1][j]; na[1][j] = na[2][j]; }
+#pragma unroll
+                for (int j = 0; j < kNB; ++j) { nbv[0][j] = nbv[1][j]; nbv[1][j] = nbv[2][j]; }
+            }
+        }
+        if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) latch_status(3 /* FP8Q_DEV_BAD_SCALES */);
+        } else if (!MX && (warp == 1 || warp == 3)) {
         // ------------------------------------------------------------ MMA issuers
         // Warp 1 issues the K groups that accumulate into TMEM buffer 0, warp 3 those into buffer
         // 1 (independent accumulators), so the issuing work is split over two SM sub-partitions.
@@ -465,14 +614,71 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
             // The row and block scales of the item's groups are pulled into L2 up front (one line
             // per group holds this warp's 32 row scales), so the per-group loads below, issued one
             // group ahead, find them there instead of in HBM.
-            for (int k = it.kb0 + 1 + lane; k < it.kb1; k += 32) {
+            for (int k = it.kb0 + 1 + lane; !MX && k < it.kb1; k += 32) {
                 prefetch_l2(args.sA + (size_t)k * args.M + min(ti.row0 + quad * 32, args.M - 1));
                 if (MODE != kModeWgrad) prefetch_l2(sb_ptr + (size_t)k * sb_step);
             }
-            float sa_next = in_a ? __ldg(sa_ptr + (size_t)it.kb0 * args.M) : 0.0f;
-            float sb_next = (MODE != kModeWgrad) ? __ldg(sb_ptr + (size_t)it.kb0 * sb_step) : 1.0f;
+            float sa_next = (!MX && in_a) ? __ldg(sa_ptr + (size_t)it.kb0 * args.M) : 0.0f;
+            float sb_next = (!MX && MODE != kModeWgrad) ? __ldg(sb_ptr + (size_t)it.kb0 * sb_step) : 1.0f;
             bool ok = true;
-            for (int kb = it.kb0; kb < it.kb1; ++kb) {
+            if (MX) {
+                // The item's whole K sits in the one TMEM accumulator: copy it into the registers
+                // (same layouts as the promotion below: a row per thread, or for Wgrad 4 rows x 2
+                // columns per 8-column block), two loads in flight, and hand the accumulator back
+                // as soon as the last load has landed.
+                if (!warp_wait(tfull_bar(0), tph, abort_flag)) {
+                    ok = false;
+                } else {
+                    tc_fence_after();
+                    const uint32_t taddr = tmem_base + lane_base + (uint32_t)(half * S::kCols);
+                    const auto tload = [&](int ch, uint32_t (&r)[kCW]) {
+                        if (MODE != kModeWgrad) {
+                            tmem_ld_async(taddr + ch * kCW, r);
+                        } else {
+                            tmem_ld_16x256b_x2(taddr + ch * kCW, r);
+                            tmem_ld_16x256b_x2(taddr + (16u << 16) + ch * kCW, r + 8);
+                        }
+                    };
+                    const auto take = [&](uint32_t (&cur)[kCW], int ch) {
+                        if (MODE != kModeWgrad) {
+#pragma unroll
+                            for (int j = 0; j < kCW; j += 2)
+                                acc[(ch * kCW + j) / 2] = make_float2(__uint_as_float(cur[j]), __uint_as_float(cur[j + 1]));
+                        } else {
+#pragma unroll
+                            for (int b = 0; b < 2; ++b)
+#pragma unroll
+                                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                                    for (int q = 0; q < 2; ++q) {
+                                        const int r0 = 8 * h + 4 * b + 2 * q;
+                                        acc[kBlocks * (2 * h + q) + 2 * ch + b] =
+                                            make_float2(__uint_as_float(cur[r0]), __uint_as_float(cur[r0 + 1]));
+                                    }
+                        }
+                    };
+                    uint32_t ra[kCW], rb[kCW];
+                    tload(0, ra);
+                    tmem_wait_ld(ra);
+#pragma unroll
+                    for (int ch = 0; ch < kChunks; ++ch) {
+                        if (ch + 1 < kChunks) {
+                            if (ch & 1) tload(ch + 1, ra);
+                            else tload(ch + 1, rb);
+                        } else {
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(tempty_bar(0));
+                        }
+                        if (ch & 1) take(rb, ch); else take(ra, ch);
+                        if (ch + 1 < kChunks) {
+                            if (ch & 1) tmem_wait_ld(ra); else tmem_wait_ld(rb);
+                        }
+                    }
+                    tph ^= 1u;
+                }
+            }
+            for (int kb = it.kb0; !MX && kb < it.kb1; ++kb) {
                 const float sa = sa_next, sbv = sb_next;
                 if (kb + 1 < it.kb1) {
                     sa_next = in_a ? __ldg(sa_ptr + (size_t)(kb + 1) * args.M) : 0.0f;
@@ -631,7 +837,7 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                         amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(h)), fabsf(bf16_hi(h))));
                     }
                     float qs;
-                    group_scale(amax, qs, qinv);
+                    group_scale<MX>(amax, qs, qinv);
                     if (row < args.M) args.s_out[(size_t)(ncol0 >> 7) * (size_t)args.M + row] = qs;
                 }
                 const bool store_d = GROUPED || MODE == kModeWgrad || args.store_d;

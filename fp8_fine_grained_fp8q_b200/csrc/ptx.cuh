@@ -263,6 +263,30 @@ __device__ __forceinline__ void mma_f8f6f4(uint32_t d_tmem, uint64_t adesc, uint
         : "memory");
 }
 
+// Block-scaled FP8 MMA (kind::mxf8f6f4, one UE8M0 scale per row of A / column of B per
+// 32-element K block): D[tmem] (+)= (A * sfA) (B * sfB)^T.  sfa_tmem / sfb_tmem address the
+// scale factors in TMEM (column, with the byte within the 32-bit column in bits 30-31, which
+// the instruction descriptor repeats as the scale-factor ids).
+__device__ __forceinline__ void mma_mxf8f6f4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+        : "memory");
+}
+
+// Asynchronous shared-memory -> TMEM copy of 32 rows x 128 bits, written to all four 32-lane
+// sub-partitions (TMEM lanes r, 32 + r, 64 + r, 96 + r get row r; 4 consecutive columns).
+// Ordered with the thread's later tcgen05.mma like any tcgen05 operation; tracked by
+// tcgen05.commit.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc)
+{
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 // Arrive once on `bar` when every tcgen05 operation issued so far by this thread completes.
 __device__ __forceinline__ void tc_commit(uint32_t bar)
 {
@@ -371,6 +395,25 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
 {
     return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16) |
            ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Shared-memory descriptor of a K-major operand without swizzling whose rows are 16 bytes:
+// core matrices of 8 rows x 16 bytes, 128 contiguous bytes each; consecutive 8-row groups
+// `sbo_bytes` apart.  A single 16-byte column needs no leading-dimension offset.  The source
+// form of tcgen05.cp 32x128b.  Layout type SWIZZLE_NONE = 0.
+__device__ __forceinline__ uint64_t sdesc_plain(uint32_t saddr, uint32_t sbo_bytes)
+{
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+
+// Instruction descriptor of kind::mxf8f6f4 with E4M3 A and B, UE8M0 scale factors, FP32
+// accumulate, M = 128: bits [4,6) B scale-factor id, [7,10) / [10,13) A / B format (E4M3 = 0),
+// 15 / 16 A / B MN-major, [17,23) N / 8, 23 scale type (UE8M0 = 1), [24,29) M / 16,
+// [29,31) A scale-factor id.
+__host__ __device__ constexpr uint32_t idesc_mx_e4m3(int n, bool b_mn_major, uint32_t sfa_id, uint32_t sfb_id)
+{
+    return (sfb_id << 4) | (0u << 7) | (0u << 10) | (0u << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+           ((uint32_t)(n >> 3) << 17) | (1u << 23) | ((uint32_t)(128 >> 4) << 24) | (sfa_id << 29);
 }
 
 // Instruction descriptor of kind::f8f6f4 with E4M3 A and B, FP32 accumulate, M = 128.

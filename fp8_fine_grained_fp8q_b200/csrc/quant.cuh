@@ -54,11 +54,24 @@ __device__ __forceinline__ uint2 quant8(const uint4& v, float inv)
     return o;
 }
 
+// POW2 = false: the max-abs scale s = a / 448.  POW2 = true (the UE8M0 variant, a separate
+// mode): s = the smallest power of two not below the binary32 quotient r = a / 448, which the
+// block-scaled tensor-core MMA can take as an 8-bit exponent; 1 / s is then an exact power of
+// two too.  r lies in [2^-109, 2^120), a normal binary32 number, so s and 1 / s are formed
+// directly from its biased exponent (rounded up when r has a nonzero fraction).
+template <bool POW2>
 __device__ __forceinline__ void group_scale(float amax, float& s, float& inv)
 {
     const float a = fmaxf(amax, kAmaxFloor);
-    s = __fdiv_rn(a, kE4M3Max);
-    inv = __fdiv_rn(kE4M3Max, a);
+    if (POW2) {
+        const uint32_t r = __float_as_uint(__fdiv_rn(a, kE4M3Max));
+        const uint32_t e = (r >> 23) + ((r & 0x7FFFFFu) != 0u ? 1u : 0u);
+        s = __uint_as_float(e << 23);
+        inv = __uint_as_float((254u - e) << 23);
+    } else {
+        s = __fdiv_rn(a, kE4M3Max);
+        inv = __fdiv_rn(kE4M3Max, a);
+    }
 }
 
 // ------------------------------------------------------------------------------------------
@@ -73,7 +86,7 @@ __device__ __forceinline__ float amax16(const uint4& a, const uint4& b)
     return fmaxf(amax8(a), amax8(b));
 }
 
-template <int UNR>
+template <int UNR, bool POW2>
 __global__ void __launch_bounds__(256) act_1x128_kernel(const uint16_t* __restrict__ x,
                                                         uint8_t* __restrict__ q,
                                                         float* __restrict__ s, int M, int K)
@@ -108,7 +121,7 @@ __global__ void __launch_bounds__(256) act_1x128_kernel(const uint16_t* __restri
 #pragma unroll
             for (int o = 4; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
             float sc, inv;
-            group_scale(amax, sc, inv);
+            group_scale<POW2>(amax, sc, inv);
             if (t < ntiles) {
                 const uint2 lo = quant8(v[u][0], inv), hi = quant8(v[u][1], inv);
                 reinterpret_cast<uint4*>(q + (size_t)t * 128)[sub] = make_uint4(lo.x, lo.y, hi.x, hi.y);
@@ -133,6 +146,7 @@ __global__ void __launch_bounds__(256) act_1x128_kernel(const uint16_t* __restri
 constexpr int kT1Tok = 128;
 constexpr int kT1Ch = 64;
 
+template <bool POW2>
 __global__ void __launch_bounds__(256) act_128x1_t_kernel(const uint16_t* __restrict__ x,
                                                           uint8_t* __restrict__ qt,
                                                           float* __restrict__ s, int64_t T, int64_t C)
@@ -166,7 +180,7 @@ __global__ void __launch_bounds__(256) act_128x1_t_kernel(const uint16_t* __rest
 #pragma unroll
         for (int k = 1; k < 8; ++k) a = fmaxf(a, red[k][threadIdx.x]);
         float sc, inv;
-        group_scale(a, sc, inv);
+        group_scale<POW2>(a, sc, inv);
         s[tb * C + c0 + threadIdx.x] = sc;
         inv_c[threadIdx.x] = inv;
     }
@@ -198,6 +212,7 @@ __global__ void __launch_bounds__(256) act_128x1_t_kernel(const uint16_t* __rest
 constexpr int kRgMaxGroups = 1024;
 constexpr int kRgChunk = 8;   // 64-channel blocks per CTA
 
+template <bool POW2>
 __global__ void __launch_bounds__(256) act_128x1_t_ragged_kernel(const uint16_t* __restrict__ x,
                                                                  const int32_t* __restrict__ offsets, int E,
                                                                  int64_t Mtot, int64_t C, uint8_t* __restrict__ qt,
@@ -279,7 +294,7 @@ __global__ void __launch_bounds__(256) act_128x1_t_ragged_kernel(const uint16_t*
 #pragma unroll
             for (int k = 1; k < 8; ++k) a = fmaxf(a, red[k][threadIdx.x]);
             float sc, inv;
-            group_scale(a, sc, inv);
+            group_scale<POW2>(a, sc, inv);
             s[(int64_t)g * C + c0 + threadIdx.x] = sc;
             inv_c[threadIdx.x] = inv;
         }
@@ -312,6 +327,7 @@ __global__ void __launch_bounds__(256) act_128x1_t_ragged_kernel(const uint16_t*
 // ------------------------------------------------------------------------------------------
 // One 128x128 tile (column block cb, token block tb) of the dual quantiser; red [8][128] and
 // inv_c [128] are this CTA's shared scratch.
+template <bool POW2>
 __device__ __forceinline__ void act_dual_tile(const uint16_t* __restrict__ x, uint8_t* __restrict__ q,
                                               float* __restrict__ s, uint8_t* __restrict__ qt,
                                               float* __restrict__ st, int64_t T, int64_t C, int64_t cb,
@@ -365,7 +381,7 @@ __device__ __forceinline__ void act_dual_tile(const uint16_t* __restrict__ x, ui
         rm[0] = fmaxf(rm[0], __shfl_xor_sync(0xFFFFFFFFu, rm[0], 1));
     }
     float rsc, rinv;
-    group_scale(rm[0], rsc, rinv);                      // row 16w + (lane >> 1)
+    group_scale<POW2>(rm[0], rsc, rinv);                      // row 16w + (lane >> 1)
     if (!(lane & 1)) s[cb * T + trow + (lane >> 1)] = rsc;
 
     __syncthreads();
@@ -374,7 +390,7 @@ __device__ __forceinline__ void act_dual_tile(const uint16_t* __restrict__ x, ui
 #pragma unroll
         for (int k = 1; k < 8; ++k) a = fmaxf(a, red[k][threadIdx.x]);
         float sc, inv;
-        group_scale(a, sc, inv);
+        group_scale<POW2>(a, sc, inv);
         st[tb * C + c0 + threadIdx.x] = sc;
         inv_c[threadIdx.x] = inv;
     }
@@ -411,6 +427,7 @@ __device__ __forceinline__ void act_dual_tile(const uint16_t* __restrict__ x, ui
         *reinterpret_cast<uint4*>(dst + (size_t)j * (size_t)T) = make_uint4(c[j][0], c[j][1], c[j][2], c[j][3]);
 }
 
+template <bool POW2>
 __global__ void __launch_bounds__(256, 3) act_dual_kernel(const uint16_t* __restrict__ x,
                                                        uint8_t* __restrict__ q, float* __restrict__ s,
                                                        uint8_t* __restrict__ qt, float* __restrict__ st,
@@ -420,7 +437,7 @@ __global__ void __launch_bounds__(256, 3) act_dual_kernel(const uint16_t* __rest
     griddep_wait();
     __shared__ __align__(16) float red[8][128];
     __shared__ __align__(16) float inv_c[128];
-    act_dual_tile(x, q, s, qt, st, T, C, blockIdx.x, blockIdx.y, red, inv_c);
+    act_dual_tile<POW2>(x, q, s, qt, st, T, C, blockIdx.x, blockIdx.y, red, inv_c);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -429,6 +446,7 @@ __global__ void __launch_bounds__(256, 3) act_dual_kernel(const uint16_t* __rest
 // ------------------------------------------------------------------------------------------
 // One 128x128 block (column block kb, row block nb) of the weight quantiser; red [8] and
 // codes [128][144] are this CTA's shared scratch (codes only when qt is requested).
+template <bool POW2>
 __device__ __forceinline__ void weight_tile(const uint16_t* __restrict__ w, uint8_t* __restrict__ q,
                                             float* __restrict__ s, uint8_t* __restrict__ qt, int64_t N,
                                             int64_t K, int64_t kb, int64_t nb, float* red,
@@ -456,7 +474,7 @@ __device__ __forceinline__ void weight_tile(const uint16_t* __restrict__ w, uint
 #pragma unroll
     for (int i = 1; i < 8; ++i) amax = fmaxf(amax, red[i]);
     float sc, inv;
-    group_scale(amax, sc, inv);
+    group_scale<POW2>(amax, sc, inv);
     if (tid == 0) s[nb * KB + kb] = sc;
 
     uint8_t* qb = q + nb * 128 * K + kb * 128;
@@ -487,6 +505,7 @@ __device__ __forceinline__ void weight_tile(const uint16_t* __restrict__ w, uint
     }
 }
 
+template <bool POW2>
 __global__ void __launch_bounds__(256) weight_128x128_kernel(const uint16_t* __restrict__ w,
                                                              uint8_t* __restrict__ q,
                                                              float* __restrict__ s,
@@ -496,7 +515,7 @@ __global__ void __launch_bounds__(256) weight_128x128_kernel(const uint16_t* __r
     griddep_wait();
     __shared__ float red[8];
     __shared__ __align__(16) uint8_t codes[128][128 + 16];
-    weight_tile(w, q, s, qt, N, K, blockIdx.x, blockIdx.y, red, codes);
+    weight_tile<POW2>(w, q, s, qt, N, K, blockIdx.x, blockIdx.y, red, codes);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -505,6 +524,7 @@ __global__ void __launch_bounds__(256) weight_128x128_kernel(const uint16_t* __r
 // takes dual tile b (token-block-major) while b < tiles_x, then weight block b - tiles_x; one
 // grid instead of two saves a launch and a partly filled last wave.
 // ------------------------------------------------------------------------------------------
+template <bool POW2>
 __global__ void __launch_bounds__(256, 3) forward_operands_kernel(
     const uint16_t* __restrict__ x, uint8_t* __restrict__ xq, float* __restrict__ xs, uint8_t* __restrict__ xqt,
     float* __restrict__ xst, int64_t T, int64_t C, const uint16_t* __restrict__ w, uint8_t* __restrict__ wq,
@@ -519,12 +539,12 @@ __global__ void __launch_bounds__(256, 3) forward_operands_kernel(
     if (b < tiles_x) {
         float (*red)[128] = reinterpret_cast<float (*)[128]>(scratch);
         float* inv_c = reinterpret_cast<float*>(scratch + 8 * 128 * 4);
-        act_dual_tile(x, xq, xs, xqt, xst, T, C, b % CB, b / CB, red, inv_c);
+        act_dual_tile<POW2>(x, xq, xs, xqt, xst, T, C, b % CB, b / CB, red, inv_c);
     } else {
         const int64_t bw = b - tiles_x;
         uint8_t (*codes)[128 + 16] = reinterpret_cast<uint8_t (*)[128 + 16]>(scratch);
         float* red = reinterpret_cast<float*>(scratch + 128 * (128 + 16));
-        weight_tile(w, wq, ws, wqt, N, C, bw % CB, bw / CB, red, codes);
+        weight_tile<POW2>(w, wq, ws, wqt, N, C, bw % CB, bw / CB, red, codes);
     }
 }
 

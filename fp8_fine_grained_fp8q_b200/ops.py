@@ -18,7 +18,9 @@ import torch
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfp8q.so")
 
 FPROP, DGRAD, WGRAD, WGRAD_ACC = 0, 1, 2, 3
-DEV_OK, DEV_TIMEOUT, DEV_BAD_OFFSETS = 0, 1, 2
+DEV_OK, DEV_TIMEOUT, DEV_BAD_OFFSETS, DEV_BAD_SCALES = 0, 1, 2, 3
+# Quantiser scale formats: the pages' max-abs scale a / 448, or the power-of-two (UE8M0) variant.
+SCALE_FORMATS = {"fp32": 0, "ue8m0": 1}
 
 _lib = None
 
@@ -56,6 +58,12 @@ def lib() -> ctypes.CDLL:
         "fp8_grouped_gemm_blockscaled_wgrad": [P, P, P, P, P, I32, I64, I64, I64, I64, P, P],
         "fp8q_act_128x1_transposed_ragged": [P, P, I32, I64, I64, P, P, I64, P],
         "fp8q_device_status": [P, ctypes.POINTER(I)],
+        "fp8q_act_1x128_fmt": [P, I64, I64, P, P, I, P],
+        "fp8q_act_128x1_transposed_fmt": [P, I64, I64, P, P, I, P],
+        "fp8q_act_dual_fmt": [P, I64, I64, P, P, P, P, I, P],
+        "fp8q_quant_forward_fmt": [P, I64, I64, P, P, P, P, P, I64, P, P, P, I, P],
+        "fp8q_weight_128x128_fmt": [P, I64, I64, P, P, P, I, P],
+        "fp8_gemm_blockscaled_ue8m0": [I, P, P, P, P, P, I64, I64, I64, P, ctypes.c_size_t, P],
     }.items():
         fn = getattr(L, name)
         fn.restype = I
@@ -107,34 +115,51 @@ def _p(t):
     return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
 
 
+def _fmt(scale_fmt: str) -> int:
+    try:
+        return SCALE_FORMATS[scale_fmt]
+    except KeyError:
+        raise ValueError(f"scale_fmt must be one of {sorted(SCALE_FORMATS)}") from None
+
+
 # ------------------------------------------------------------------------------------------ #
 # Quantisers
 # ------------------------------------------------------------------------------------------ #
 
-def act_1x128(x: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tensor | None = None):
-    """x[M,K] bf16 -> (q[M,K] uint8 E4M3 codes, s[K/128, M] fp32)."""
+def act_1x128(x: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tensor | None = None,
+              scale_fmt: str = "fp32"):
+    """x[M,K] bf16 -> (q[M,K] uint8 E4M3 codes, s[K/128, M] fp32).  scale_fmt "ue8m0" selects the
+    power-of-two scales (fp8q_act_1x128_fmt)."""
     _require(x, "x", torch.bfloat16, 2)
     M, K = x.shape
     q = _out(q, (M, K), torch.uint8, x.device, "q")
     s = _out(s, (K // 128, M), torch.float32, x.device, "s")
-    _check("fp8q_act_1x128", lib().fp8q_act_1x128(_p(x), M, K, _p(q), _p(s), _stream(x.device)))
+    if scale_fmt == "fp32":
+        _check("fp8q_act_1x128", lib().fp8q_act_1x128(_p(x), M, K, _p(q), _p(s), _stream(x.device)))
+    else:
+        _check("fp8q_act_1x128_fmt", lib().fp8q_act_1x128_fmt(_p(x), M, K, _p(q), _p(s), _fmt(scale_fmt),
+                                                              _stream(x.device)))
     return q, s
 
 
 def act_128x1_transposed(x: torch.Tensor, qt: torch.Tensor | None = None,
-                         s: torch.Tensor | None = None):
+                         s: torch.Tensor | None = None, scale_fmt: str = "fp32"):
     """x[T,C] bf16 -> (qt[C,T] uint8, s[T/128, C] fp32)."""
     _require(x, "x", torch.bfloat16, 2)
     T, C = x.shape
     qt = _out(qt, (C, T), torch.uint8, x.device, "qt")
     s = _out(s, (T // 128, C), torch.float32, x.device, "s")
-    _check("fp8q_act_128x1_transposed",
-           lib().fp8q_act_128x1_transposed(_p(x), T, C, _p(qt), _p(s), _stream(x.device)))
+    if scale_fmt == "fp32":
+        _check("fp8q_act_128x1_transposed",
+               lib().fp8q_act_128x1_transposed(_p(x), T, C, _p(qt), _p(s), _stream(x.device)))
+    else:
+        _check("fp8q_act_128x1_transposed_fmt",
+               lib().fp8q_act_128x1_transposed_fmt(_p(x), T, C, _p(qt), _p(s), _fmt(scale_fmt), _stream(x.device)))
     return qt, s
 
 
 def act_dual(x: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tensor | None = None,
-             qt: torch.Tensor | None = None, st: torch.Tensor | None = None):
+             qt: torch.Tensor | None = None, st: torch.Tensor | None = None, scale_fmt: str = "fp32"):
     """x[T,C] bf16 -> (q[T,C], s[C/128, T], qt[C,T], st[T/128, C]) in one pass over x: the
     outputs of act_1x128(x) and act_128x1_transposed(x), bit for bit."""
     _require(x, "x", torch.bfloat16, 2)
@@ -143,13 +168,18 @@ def act_dual(x: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tensor | N
     s = _out(s, (C // 128, T), torch.float32, x.device, "s")
     qt = _out(qt, (C, T), torch.uint8, x.device, "qt")
     st = _out(st, (T // 128, C), torch.float32, x.device, "st")
-    _check("fp8q_act_dual",
-           lib().fp8q_act_dual(_p(x), T, C, _p(q), _p(s), _p(qt), _p(st), _stream(x.device)))
+    if scale_fmt == "fp32":
+        _check("fp8q_act_dual",
+               lib().fp8q_act_dual(_p(x), T, C, _p(q), _p(s), _p(qt), _p(st), _stream(x.device)))
+    else:
+        _check("fp8q_act_dual_fmt",
+               lib().fp8q_act_dual_fmt(_p(x), T, C, _p(q), _p(s), _p(qt), _p(st), _fmt(scale_fmt),
+                                       _stream(x.device)))
     return q, s, qt, st
 
 
 def quant_forward(x: torch.Tensor, w: torch.Tensor, xq=None, xs=None, xqt=None, xst=None,
-                  wq=None, ws=None, wqt=None, transposed_w: bool = False):
+                  wq=None, ws=None, wqt=None, transposed_w: bool = False, scale_fmt: str = "fp32"):
     """x[T,C], w[N,C] bf16 -> ((xq, xs, xqt, xst), (wq, ws, wqt or None)) in one launch: the outputs of
     act_dual(x) and weight_128x128(w), bit for bit."""
     _require(x, "x", torch.bfloat16, 2)
@@ -167,14 +197,19 @@ def quant_forward(x: torch.Tensor, w: torch.Tensor, xq=None, xs=None, xqt=None, 
     ws = _out(ws, (N // 128, C // 128), torch.float32, dev, "ws")
     if transposed_w or wqt is not None:
         wqt = _out(wqt, (C, N), torch.uint8, dev, "wqt")
-    _check("fp8q_quant_forward",
-           lib().fp8q_quant_forward(_p(x), T, C, _p(xq), _p(xs), _p(xqt), _p(xst), _p(w), N, _p(wq), _p(ws),
-                                    _p(wqt), _stream(dev)))
+    if scale_fmt == "fp32":
+        _check("fp8q_quant_forward",
+               lib().fp8q_quant_forward(_p(x), T, C, _p(xq), _p(xs), _p(xqt), _p(xst), _p(w), N, _p(wq), _p(ws),
+                                        _p(wqt), _stream(dev)))
+    else:
+        _check("fp8q_quant_forward_fmt",
+               lib().fp8q_quant_forward_fmt(_p(x), T, C, _p(xq), _p(xs), _p(xqt), _p(xst), _p(w), N, _p(wq),
+                                            _p(ws), _p(wqt), _fmt(scale_fmt), _stream(dev)))
     return (xq, xs, xqt, xst), (wq, ws, wqt)
 
 
 def weight_128x128(w: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tensor | None = None,
-                   transposed: bool = False, qt: torch.Tensor | None = None):
+                   transposed: bool = False, qt: torch.Tensor | None = None, scale_fmt: str = "fp32"):
     """w[N,K] bf16 -> (q[N,K] uint8, s[N/128, K/128] fp32, qt[K,N] uint8 or None)."""
     _require(w, "w", torch.bfloat16, 2)
     N, K = w.shape
@@ -182,8 +217,12 @@ def weight_128x128(w: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tens
     s = _out(s, (N // 128, K // 128), torch.float32, w.device, "s")
     if transposed or qt is not None:
         qt = _out(qt, (K, N), torch.uint8, w.device, "qt")
-    _check("fp8q_weight_128x128",
-           lib().fp8q_weight_128x128(_p(w), N, K, _p(q), _p(s), _p(qt), _stream(w.device)))
+    if scale_fmt == "fp32":
+        _check("fp8q_weight_128x128",
+               lib().fp8q_weight_128x128(_p(w), N, K, _p(q), _p(s), _p(qt), _stream(w.device)))
+    else:
+        _check("fp8q_weight_128x128_fmt",
+               lib().fp8q_weight_128x128_fmt(_p(w), N, K, _p(q), _p(s), _p(qt), _fmt(scale_fmt), _stream(w.device)))
     return q, s, qt
 
 
@@ -209,7 +248,7 @@ def gemm_workspace(mode: int, M: int, N: int, K: int, device: torch.device) -> t
 
 def gemm_blockscaled(mode: int, A: torch.Tensor, sA: torch.Tensor, B: torch.Tensor,
                      sB: torch.Tensor, out: torch.Tensor | None = None,
-                     workspace: torch.Tensor | None = None):
+                     workspace: torch.Tensor | None = None, _entry: str = "fp8_gemm_blockscaled"):
     """Block-scaled FP8 GEMM.  FPROP: B = W[N,K]; DGRAD: B = W[K,N]; WGRAD: B = X^T[N,K];
     WGRAD_ACC: as WGRAD, added into `out` (required, fp32).
     Returns D[M,N] (bf16, or fp32 for WGRAD / WGRAD_ACC).  `workspace` (uint8, CUDA) enables the
@@ -231,10 +270,20 @@ def gemm_blockscaled(mode: int, A: torch.Tensor, sA: torch.Tensor, B: torch.Tens
     if workspace is None:
         workspace = gemm_workspace(mode, M, N, K, A.device)
     ws_ptr, ws_bytes = (None, 0) if workspace is None else (_p(workspace), workspace.numel())
-    _check("fp8_gemm_blockscaled",
-           lib().fp8_gemm_blockscaled(int(mode), _p(A), _p(sA), _p(B), _p(sB), _p(out), M, N, K,
-                                      ws_ptr, ws_bytes, _stream(A.device)))
+    _check(_entry, getattr(lib(), _entry)(int(mode), _p(A), _p(sA), _p(B), _p(sB), _p(out), M, N, K,
+                                          ws_ptr, ws_bytes, _stream(A.device)))
     return out
+
+
+def gemm_blockscaled_ue8m0(mode: int, A: torch.Tensor, sA: torch.Tensor, B: torch.Tensor,
+                           sB: torch.Tensor, out: torch.Tensor | None = None,
+                           workspace: torch.Tensor | None = None):
+    """The GEMM of gemm_blockscaled for power-of-two scales (the scale_fmt="ue8m0" quantisers'):
+    the tensor core applies them inside the MMA (tcgen05 kind::mxf8f6f4) and accumulates the
+    whole K in FP32.  Same arguments and layouts; a scale that is not a power of two latches
+    DEV_BAD_SCALES (see device_status)."""
+    return gemm_blockscaled(mode, A, sA, B, sB, out=out, workspace=workspace,
+                            _entry="fp8_gemm_blockscaled_ue8m0")
 
 
 def gemm_blockscaled_quant(mode: int, A: torch.Tensor, sA: torch.Tensor, B: torch.Tensor,

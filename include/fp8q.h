@@ -71,7 +71,15 @@ enum {
 enum {
     FP8Q_DEV_OK = 0,
     FP8Q_DEV_TIMEOUT = 1,      /* a bounded pipeline wait expired; the kernel exited early */
-    FP8Q_DEV_BAD_OFFSETS = 2   /* grouped GEMM: offsets not 0-based / nondecreasing / ending at Mtot */
+    FP8Q_DEV_BAD_OFFSETS = 2,  /* grouped GEMM: offsets not 0-based / nondecreasing / ending at Mtot */
+    FP8Q_DEV_BAD_SCALES = 3    /* fp8_gemm_blockscaled_ue8m0: a scale that is not a positive normal
+                                  power of two (its result is then unspecified) */
+};
+
+/* Scale formats of the quantisers (the *_fmt entry points). */
+enum {
+    FP8Q_SCALE_FP32 = 0,       /* s = a / 448, the pages' max-abs scale (all other entry points) */
+    FP8Q_SCALE_UE8M0 = 1       /* s = the smallest power of two >= fl32(a / 448): see below */
 };
 
 /* GEMM modes (the three GEMMs of a linear layer, [REPOST] paragraph 2, Figure 6; the FP32
@@ -277,6 +285,45 @@ FP8Q_API int fp8q_act_128x1_transposed_ragged(const uint16_t* x, const int32_t* 
 FP8Q_API int fp8_grouped_gemm_blockscaled_wgrad(const uint8_t* A, const float* sA, const uint8_t* B, const float* sB,
                                                 const int32_t* offsets, int32_t E, int64_t Mtot, int64_t M, int64_t N,
                                                 int64_t Kcap, float* D, fp8q_stream_t stream);
+
+/*
+ * Power-of-two (UE8M0) scale variant.  A separate mode with its own scale semantics, not one the
+ * pages describe: the block-scaled tensor-core MMA of sm_100a (tcgen05.mma kind::mxf8f6f4) takes
+ * per-32-element scales as 8-bit exponents (UE8M0) and applies them inside the MMA, so the GEMM
+ * accumulates the whole K in the tensor core's FP32 accumulator with no per-128-K promotion.
+ * Groups stay 1x128, 128x1 and 128x128; only the scale of a group changes:
+ *   a = max(max|x| over g, 2^-100);  r = a / 448 (binary32, round to nearest);
+ *   s = the smallest power of two >= r (stored as an fp32 value, exactly a power of two);
+ *   q = E4M3(x * (1 / s)), 1 / s an exact power of two.
+ * The *_fmt quantisers take scale_fmt = FP8Q_SCALE_FP32 (identical to the entry point without
+ * the suffix) or FP8Q_SCALE_UE8M0; other arguments, layouts and errors as those entry points
+ * (FP8Q_ERR_ARG for an unknown scale_fmt).
+ */
+FP8Q_API int fp8q_act_1x128_fmt(const uint16_t* x, int64_t M, int64_t K, uint8_t* q, float* s, int scale_fmt,
+                                fp8q_stream_t stream);
+FP8Q_API int fp8q_act_128x1_transposed_fmt(const uint16_t* x, int64_t T, int64_t C, uint8_t* qt, float* s,
+                                           int scale_fmt, fp8q_stream_t stream);
+FP8Q_API int fp8q_act_dual_fmt(const uint16_t* x, int64_t T, int64_t C, uint8_t* q, float* s, uint8_t* qt,
+                               float* st, int scale_fmt, fp8q_stream_t stream);
+FP8Q_API int fp8q_quant_forward_fmt(const uint16_t* x, int64_t T, int64_t C, uint8_t* xq, float* xs, uint8_t* xqt,
+                                    float* xst, const uint16_t* w, int64_t N, uint8_t* wq, float* ws,
+                                    uint8_t* wqt_or_null, int scale_fmt, fp8q_stream_t stream);
+FP8Q_API int fp8q_weight_128x128_fmt(const uint16_t* w, int64_t N, int64_t K, uint8_t* q, float* s,
+                                     uint8_t* qt_or_null, int scale_fmt, fp8q_stream_t stream);
+
+/*
+ * Block-scaled FP8 GEMM for power-of-two scales: D = sum_k A^(m, k) B^(k, n) with the dequantised
+ * operands A^ = dec(A) sA, B^ = dec(B) sB, computed by tcgen05.mma kind::mxf8f6f4 with each
+ * 128-group's scale exponent replicated over its four 32-element blocks; the products are exact
+ * and the whole K is accumulated in FP32 by the tensor core.  Arguments, operand layouts,
+ * modes (FP8Q_FPROP, FP8Q_DGRAD, FP8Q_WGRAD, FP8Q_WGRAD_ACC), requirements, workspace and return
+ * codes exactly as fp8_gemm_blockscaled, except that every scale read must be a positive normal
+ * power of two (the FP8Q_SCALE_UE8M0 quantisers produce only such scales); any other scale latches
+ * FP8Q_DEV_BAD_SCALES and leaves D unspecified.  Scales of rows past M are not read.
+ */
+FP8Q_API int fp8_gemm_blockscaled_ue8m0(int mode, const uint8_t* A, const float* sA, const uint8_t* B,
+                                        const float* sB, void* D, int64_t M, int64_t N, int64_t K,
+                                        void* workspace, size_t ws_bytes, fp8q_stream_t stream);
 
 /*
  * Synchronise `stream`, then read and clear the device status word of the current device.

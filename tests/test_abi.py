@@ -33,7 +33,7 @@ def test_header_declares_the_boundary():
     names = set(declared_symbols())
     assert {"fp8q_act_1x128", "fp8q_act_128x1_transposed", "fp8q_weight_128x128",
             "fp8_gemm_blockscaled", "fp8_grouped_gemm_blockscaled", "fp8q_device_status",
-            "fp8q_status_string"} <= names
+            "fp8q_status_string", "fp8_gemm_blockscaled_ue8m0", "fp8q_act_1x128_fmt"} <= names
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -119,6 +119,32 @@ def test_gemm_host_checks(L):
     # Stream-K workspace: one 128 x 256 FP32 slot per CTA plus flags; none for a single K group.
     assert L.fp8q_gemm_workspace_size(0, 4096, 2048, 7168) >= 148 * 128 * 256 * 4
     assert L.fp8q_gemm_workspace_size(0, 4096, 2048, 128) == 0
+
+
+def test_ue8m0_entries_host_checks(L):
+    s = None
+    g = L.fp8_gemm_blockscaled_ue8m0
+    args = (P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE))
+    assert g(5, *args, 128, 128, 128, None, 0, s) == ERR_ARG             # bad mode
+    assert g(3, *args, 128, 128, 0, None, 0, s) == OK                    # D += nothing
+    assert g(0, *args, 128, 100, 128, None, 0, s) == ERR_SHAPE
+    assert g(2, *args, 0, 128, 128, None, 0, s) == OK                    # empty
+    assert g(0, P(FAKE), None, P(FAKE), P(FAKE), P(FAKE), 128, 128, 128, None, 0, s) == ERR_ARG
+    assert g(0, P(FAKE), P(FAKE), P(FAKE), P(MISALIGNED), P(FAKE), 128, 128, 128, None, 0, s) == ERR_ALIGN
+    # The scale-format quantisers: an unknown format is an argument error; sizes as before.
+    assert L.fp8q_act_1x128_fmt(P(FAKE), 4, 128, P(FAKE), P(FAKE), 2, s) == ERR_ARG
+    assert L.fp8q_act_1x128_fmt(P(FAKE), 4, 100, P(FAKE), P(FAKE), 1, s) == ERR_SHAPE
+    assert L.fp8q_act_1x128_fmt(P(FAKE), 0, 128, P(FAKE), P(FAKE), 1, s) == OK
+    assert L.fp8q_act_128x1_transposed_fmt(P(FAKE), 128, 64, P(FAKE), P(FAKE), -1, s) == ERR_ARG
+    assert L.fp8q_act_128x1_transposed_fmt(P(FAKE), 100, 64, P(FAKE), P(FAKE), 1, s) == ERR_SHAPE
+    assert L.fp8q_act_dual_fmt(P(FAKE), 128, 128, P(FAKE), P(FAKE), P(FAKE), P(FAKE), 7, s) == ERR_ARG
+    assert L.fp8q_act_dual_fmt(P(FAKE), 128, 64, P(FAKE), P(FAKE), P(FAKE), P(FAKE), 1, s) == ERR_SHAPE
+    assert L.fp8q_quant_forward_fmt(P(FAKE), 128, 128, P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE), 128,
+                                    P(FAKE), P(FAKE), None, 9, s) == ERR_ARG
+    assert L.fp8q_weight_128x128_fmt(P(FAKE), 128, 128, P(FAKE), P(FAKE), None, 3, s) == ERR_ARG
+    assert L.fp8q_weight_128x128_fmt(P(FAKE), 128, 130, P(FAKE), P(FAKE), None, 1, s) == ERR_SHAPE
+    with pytest.raises(ValueError):
+        ops._fmt("e4m3")
 
 
 def test_gemm_quant_host_checks(L):
