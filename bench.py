@@ -224,6 +224,56 @@ def op_work():
     }
 
 
+def run_ue8m0_variant(ops, torch, t, b, flush_l2, steps):
+    """Not the headline: the same five-launch step with power-of-two (UE8M0) scales, whose GEMMs
+    run on the block-scaled tensor-core MMA without per-128-K promotion (a separate mode, not the
+    pages' method).  Whole steps with an event on each side, then each launch alone."""
+    launches = {
+        "quant_forward_XW": lambda: ops.quant_forward(t["X"], t["W"], b["Xq"], b["sX"], b["Xtq"], b["sXt"],
+                                                      b["Wq"], b["sW"], scale_fmt="ue8m0"),
+        "gemm_fprop": lambda: ops.gemm_blockscaled_ue8m0(ops.FPROP, b["Xq"], b["sX"], b["Wq"], b["sW"], b["Y"]),
+        "act_dual_dY": lambda: ops.act_dual(t["dY"], b["dYq"], b["sdY"], b["dYtq"], b["sdYt"], scale_fmt="ue8m0"),
+        "gemm_dgrad": lambda: ops.gemm_blockscaled_ue8m0(ops.DGRAD, b["dYq"], b["sdY"], b["Wq"], b["sW"], b["dX"]),
+        "gemm_wgrad": lambda: ops.gemm_blockscaled_ue8m0(ops.WGRAD, b["dYtq"], b["sdYt"], b["Xtq"], b["sXt"], b["dW"]),
+    }
+    fs = list(launches.values())
+    for _ in range(3):
+        flush_l2()
+        for f in fs:
+            f()
+    n = max(5, min(steps, 30))
+    step_ms, per = [], {k: [] for k in launches}
+    for _ in range(n):
+        flush_l2()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for f in fs:
+            f()
+        e1.record()
+        torch.cuda.synchronize()
+        step_ms.append(e0.elapsed_time(e1))
+    for _ in range(n):
+        flush_l2()
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(fs) + 1)]
+        evs[0].record()
+        for i, f in enumerate(fs):
+            f()
+            evs[i + 1].record()
+        torch.cuda.synchronize()
+        for i, k in enumerate(launches):
+            per[k].append(evs[i].elapsed_time(evs[i + 1]))
+    status = ops.device_status()
+    if status != ops.DEV_OK:
+        raise RuntimeError(f"device status {status} in the UE8M0 variant")
+    ms = statistics.median(step_ms)
+    kern = {k: round(statistics.median(v), 5) for k, v in per.items()}
+    return {"step_ms": round(ms, 5), "step_TFLOP/s": round(STEP_FLOP / (ms * 1e-3) / 1e12, 1),
+            "kernels_ms": kern,
+            "gemm_TFLOP/s": {k: round(GEMM_FLOP / (kern[k] * 1e-3) / 1e12, 1)
+                             for k in ("gemm_fprop", "gemm_dgrad", "gemm_wgrad")},
+            "steps": n, "scales": "power of two (UE8M0); tcgen05.mma kind::mxf8f6f4, whole-K TMEM accumulation"}
+
+
 def run_ours(args, rank, world, dist):
     import torch
     from fp8_fine_grained_fp8q_b200 import ops
@@ -351,6 +401,8 @@ def run_ours(args, rank, world, dist):
     e2e_sum = max_over_ranks(e2e_sum, dist, dev)
     e2e_value = world * STEP_FLOP / (e2e_sum / len(e2e_ms) * 1e-3) / 1e12
 
+    ue8m0 = run_ue8m0_variant(ops, torch, t, b, flush_l2, args.steps)
+
     peaks, peak_kind = load_peaks()
     fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
     hbm = peaks["hbm_gbs"]
@@ -394,6 +446,7 @@ def run_ours(args, rank, world, dist):
                        "hbm_peak_gbs": hbm, "peak_source": peak_kind},
         "kernels": kernels,
         "fused_output_quant_ms": fused_ms,
+        "ue8m0_variant": ue8m0,
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "steps": len(e2e_ms)},
         "gpu_launches": len(launches) * args.steps,
@@ -652,6 +705,27 @@ def run_moe(args, rank, world, dist):
     }
 
 
+def profile_gemms(fmt: str):
+    """The linear layer's three GEMMs, one launch each, after one quantisation pass (for a profiler
+    capture: `-k regex:gemm_blockscaled -c 3` takes exactly these launches)."""
+    import torch
+    from fp8_fine_grained_fp8q_b200 import ops
+    dev = torch.device("cuda", 0)
+    _, t, b = make_buffers(torch, dev)
+    ops.quant_forward(t["X"], t["W"], b["Xq"], b["sX"], b["Xtq"], b["sXt"], b["Wq"], b["sW"], scale_fmt=fmt)
+    ops.act_dual(t["dY"], b["dYq"], b["sdY"], b["dYtq"], b["sdYt"], scale_fmt=fmt)
+    gemm = ops.gemm_blockscaled if fmt == "fp32" else ops.gemm_blockscaled_ue8m0
+    torch.cuda.synchronize()
+    gemm(ops.FPROP, b["Xq"], b["sX"], b["Wq"], b["sW"], b["Y"])
+    gemm(ops.DGRAD, b["dYq"], b["sdY"], b["Wq"], b["sW"], b["dX"])
+    gemm(ops.WGRAD, b["dYtq"], b["sdYt"], b["Xtq"], b["sXt"], b["dW"])
+    torch.cuda.synchronize()
+    status = ops.device_status(dev)
+    if status != ops.DEV_OK:
+        raise RuntimeError(f"device status {status}")
+    print(json.dumps({"profile_gemms": fmt, "status": "ok"}))
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -664,7 +738,13 @@ def main():
                     help="linear: the FP8 linear layer (the headline); moe: the grouped MoE Fprop")
     ap.add_argument("--separate-quant", action="store_true",
                     help="quantise X and dY with separate 1x128 and 128x1 launches")
+    ap.add_argument("--profile-gemms", choices=["fp32", "ue8m0"], default=None,
+                    help="no timing: quantise the layer once with this scale format, launch its Fprop, "
+                         "Dgrad and Wgrad GEMMs once each and exit (a small, fixed launch list for ncu)")
     args = ap.parse_args()
+    if args.profile_gemms:
+        profile_gemms(args.profile_gemms)
+        return
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be at least 3")
 
