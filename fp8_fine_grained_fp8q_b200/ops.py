@@ -246,14 +246,9 @@ def gemm_workspace(mode: int, M: int, N: int, K: int, device: torch.device) -> t
     return ws
 
 
-def gemm_blockscaled(mode: int, A: torch.Tensor, sA: torch.Tensor, B: torch.Tensor,
-                     sB: torch.Tensor, out: torch.Tensor | None = None,
-                     workspace: torch.Tensor | None = None, _entry: str = "fp8_gemm_blockscaled"):
-    """Block-scaled FP8 GEMM.  FPROP: B = W[N,K]; DGRAD: B = W[K,N]; WGRAD: B = X^T[N,K];
-    WGRAD_ACC: as WGRAD, added into `out` (required, fp32).
-    Returns D[M,N] (bf16, or fp32 for WGRAD / WGRAD_ACC).  `workspace` (uint8, CUDA) enables the
-    stream-K schedule; by default a per-device workspace sized by fp8q_gemm_workspace_size is
-    used.  A workspace must not be shared by GEMMs that may run concurrently."""
+def _gemm(entry: str, mode: int, A: torch.Tensor, sA: torch.Tensor, B: torch.Tensor, sB: torch.Tensor,
+          out: torch.Tensor | None, workspace: torch.Tensor | None):
+    """Shared marshalling of fp8_gemm_blockscaled and fp8_gemm_blockscaled_ue8m0 (same arguments)."""
     if mode == WGRAD_ACC and out is None:
         raise ValueError("WGRAD_ACC accumulates into `out`: pass the fp32 gradient to add to")
     _require(A, "A", torch.uint8, 2)
@@ -270,9 +265,20 @@ def gemm_blockscaled(mode: int, A: torch.Tensor, sA: torch.Tensor, B: torch.Tens
     if workspace is None:
         workspace = gemm_workspace(mode, M, N, K, A.device)
     ws_ptr, ws_bytes = (None, 0) if workspace is None else (_p(workspace), workspace.numel())
-    _check(_entry, getattr(lib(), _entry)(int(mode), _p(A), _p(sA), _p(B), _p(sB), _p(out), M, N, K,
-                                          ws_ptr, ws_bytes, _stream(A.device)))
+    _check(entry, getattr(lib(), entry)(int(mode), _p(A), _p(sA), _p(B), _p(sB), _p(out), M, N, K,
+                                        ws_ptr, ws_bytes, _stream(A.device)))
     return out
+
+
+def gemm_blockscaled(mode: int, A: torch.Tensor, sA: torch.Tensor, B: torch.Tensor,
+                     sB: torch.Tensor, out: torch.Tensor | None = None,
+                     workspace: torch.Tensor | None = None):
+    """Block-scaled FP8 GEMM.  FPROP: B = W[N,K]; DGRAD: B = W[K,N]; WGRAD: B = X^T[N,K];
+    WGRAD_ACC: as WGRAD, added into `out` (required, fp32).
+    Returns D[M,N] (bf16, or fp32 for WGRAD / WGRAD_ACC).  `workspace` (uint8, CUDA) enables the
+    stream-K schedule; by default a per-device workspace sized by fp8q_gemm_workspace_size is
+    used.  A workspace must not be shared by GEMMs that may run concurrently."""
+    return _gemm("fp8_gemm_blockscaled", mode, A, sA, B, sB, out, workspace)
 
 
 def gemm_blockscaled_ue8m0(mode: int, A: torch.Tensor, sA: torch.Tensor, B: torch.Tensor,
@@ -282,8 +288,7 @@ def gemm_blockscaled_ue8m0(mode: int, A: torch.Tensor, sA: torch.Tensor, B: torc
     the tensor core applies them inside the MMA (tcgen05 kind::mxf8f6f4) and accumulates the
     whole K in FP32.  Same arguments and layouts; a scale that is not a power of two latches
     DEV_BAD_SCALES (see device_status)."""
-    return gemm_blockscaled(mode, A, sA, B, sB, out=out, workspace=workspace,
-                            _entry="fp8_gemm_blockscaled_ue8m0")
+    return _gemm("fp8_gemm_blockscaled_ue8m0", mode, A, sA, B, sB, out, workspace)
 
 
 def gemm_blockscaled_quant(mode: int, A: torch.Tensor, sA: torch.Tensor, B: torch.Tensor,
