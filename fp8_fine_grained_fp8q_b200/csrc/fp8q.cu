@@ -181,27 +181,36 @@ size_t sk_workspace_bytes(int ctas, int bn)
 }
 
 // Launch stamps: a flag holds the stamp of the launch that published it, so flags are never
-// reset.  The high half is random per process (stale workspace contents cannot match by
-// accident), the low half counts launches.
+// reset.  Bits 40..63 are a nonzero random salt drawn once per process (workspace memory left by
+// another process cannot match by accident); bits 0..39 count this process's stream-K launches
+// from 1.  Stamps are nonzero and never repeat within a process until 2^40 launches (about 35
+// years at one launch per millisecond).
 unsigned long long next_stamp()
 {
     static std::atomic<unsigned long long> counter{0};
     static const unsigned long long salt = [] {
         std::random_device rd;
         unsigned long long v = ((unsigned long long)rd() << 32) ^ (unsigned long long)rd();
-        return v | 1ull;
+        v &= 0xFFFFFFull;
+        return v ? v : 1ull;
     }();
-    return (salt & 0xFFFFFFFF00000000ull) | ((++counter) & 0xFFFFFFFFull) | 1ull << 31;
+    return (salt << 40) | ((++counter) & 0xFFFFFFFFFFull);
+}
+
+// FP8Q_GEMM_SCHED=dp / sk forces the data-parallel / stream-K schedule (tests and tuning).
+bool streamk_forced()
+{
+    const char* env = getenv("FP8Q_GEMM_SCHED");
+    return env && strcmp(env, "sk") == 0;
 }
 
 // Stream-K pays off when the tiles do not fill whole waves of the persistent grid.
-// FP8Q_GEMM_SCHED=dp / sk forces the data-parallel / stream-K schedule.
 bool want_streamk(int64_t tiles, int ctas, int kb)
 {
     const char* env = getenv("FP8Q_GEMM_SCHED");
     if (env && strcmp(env, "dp") == 0) return false;
     if (kb < 2) return false;
-    if (env && strcmp(env, "sk") == 0) return true;
+    if (streamk_forced()) return true;
     return tiles % ctas != 0;
 }
 
@@ -572,11 +581,13 @@ int fp8_gemm_blockscaled_noalloc(int mode, const uint8_t* A, const float* sA, co
                                  void* D, int64_t M, int64_t N, int64_t K, fp8q_stream_t stream)
 {
     // The stream-K schedule needs one slot per persistent CTA (one per SM); the data-parallel
-    // schedule needs none.  Refuse problems whose scratch would not fit the fixed array.
+    // schedule needs none.  When the slots would not fit the fixed array (more SMs than it was
+    // sized for) the call runs data-parallel, unless stream-K is forced.
     const size_t need = fp8q_gemm_workspace_size(mode, M, N, K);
-    if (need > kNoallocScratchBytes) return FP8Q_ERR_SCRATCH;
     void* scratch = nullptr;
-    if (need > 0) {
+    if (need > kNoallocScratchBytes) {
+        if (streamk_forced()) return FP8Q_ERR_SCRATCH;
+    } else if (need > 0) {
         scratch = noalloc_scratch();
         if (!scratch) return FP8Q_ERR_CUDA;
     }

@@ -234,14 +234,20 @@ _workspaces: dict = {}
 
 
 def gemm_workspace(mode: int, M: int, N: int, K: int, device: torch.device) -> torch.Tensor | None:
-    """The stream-K workspace a call of this size may use (cached per device; None if not needed)."""
+    """The stream-K workspace a call of this size may use (None if not needed).
+
+    Cached per (device, current stream): calls queued on one stream run one after another and may
+    share a workspace, calls on different streams may overlap on the GPU and get their own.  The
+    cache holds the tensor, so a stream's workspace lives as long as the process (or until a
+    larger call replaces it)."""
     nbytes = int(lib().fp8q_gemm_workspace_size(int(mode), M, N, K))
     if nbytes == 0:
         return None
-    key = device.index if device.index is not None else torch.cuda.current_device()
+    index = device.index if device.index is not None else torch.cuda.current_device()
+    key = (index, torch.cuda.current_stream(index).cuda_stream)
     ws = _workspaces.get(key)
     if ws is None or ws.numel() < nbytes:
-        ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=torch.device("cuda", index))
         _workspaces[key] = ws
     return ws
 
@@ -276,8 +282,9 @@ def gemm_blockscaled(mode: int, A: torch.Tensor, sA: torch.Tensor, B: torch.Tens
     """Block-scaled FP8 GEMM.  FPROP: B = W[N,K]; DGRAD: B = W[K,N]; WGRAD: B = X^T[N,K];
     WGRAD_ACC: as WGRAD, added into `out` (required, fp32).
     Returns D[M,N] (bf16, or fp32 for WGRAD / WGRAD_ACC).  `workspace` (uint8, CUDA) enables the
-    stream-K schedule; by default a per-device workspace sized by fp8q_gemm_workspace_size is
-    used.  A workspace must not be shared by GEMMs that may run concurrently."""
+    stream-K schedule; by default one workspace per (device, stream), sized by
+    fp8q_gemm_workspace_size, is used.  A workspace passed explicitly must not be shared by GEMMs
+    that may run concurrently."""
     return _gemm("fp8_gemm_blockscaled", mode, A, sA, B, sB, out, workspace)
 
 

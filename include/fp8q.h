@@ -64,7 +64,7 @@ enum {
     FP8Q_ERR_CUDA = 4,         /* a CUDA runtime or driver call failed (no device, launch error) */
     FP8Q_ERR_UNSUPPORTED = 5,  /* a size beyond what this build supports (see each call) */
     FP8Q_ERR_DEVICE = 6,       /* reported by fp8q_device_status: an error latched on the device */
-    FP8Q_ERR_SCRATCH = 7       /* fp8_gemm_blockscaled_noalloc: scratch need exceeds its fixed array */
+    FP8Q_ERR_SCRATCH = 7       /* fp8_gemm_blockscaled_noalloc with stream-K forced: scratch need exceeds its fixed array */
 };
 
 /* Device status word values (what fp8q_device_status writes to *out). */
@@ -210,9 +210,10 @@ FP8Q_API int fp8_gemm_blockscaled_quant(int mode, const uint8_t* A, const float*
  * Same arguments, results and requirements as fp8_gemm_blockscaled.  The stream-K scratch that
  * call would take from `workspace` comes instead from a fixed device array inside the library:
  * room for the partial slots and flags of 160 persistent CTAs of 256-wide tiles, about 20 MiB,
- * held by every GPU that loads the library until the process exits.  Problems whose scratch
- * would exceed it (a device with more than 160 SMs) get FP8Q_ERR_SCRATCH.  No call allocates or
- * frees anything.
+ * held by every GPU that loads the library until the process exits.  Where the slots would not
+ * fit it (a device with more than 160 SMs) the call runs the data-parallel schedule, which needs
+ * no scratch; only with stream-K forced (FP8Q_GEMM_SCHED=sk) does it return FP8Q_ERR_SCRATCH
+ * instead.  No call allocates or frees anything.
  * - The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
  *   that device current) and caches it; make that first call before any stream capture.
  * - Every call shares the one array per device and leaves its contents behind.  Nothing in it

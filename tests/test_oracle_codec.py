@@ -103,3 +103,21 @@ def test_cross_check_torch_ties():
                           np.nextafter(mid, np.float32(0))])
     pts = np.concatenate([pts, -pts])
     assert np.array_equal(oracle.e4m3_encode(pts), _torch_codes(pts))
+
+
+def test_exhaustive_binary32_against_torch():
+    """Every binary32 bit pattern with |x| <= 464 (both signs, zeros, subnormals): the oracle's
+    encoder agrees with PyTorch's float8_e4m3fn cast.  Up to 464 the nearest-even rounding of
+    either encoder never needs saturation (464 is the tie between 448 and the first value past
+    the E4M3 range, and it rounds to the even code 448), so the two must be identical."""
+    top = int(np.array([464.0], dtype=np.float32).view(np.uint32)[0])   # 0x43E80000
+    chunk = 1 << 24
+    for sign in (0, 0x80000000):
+        for lo in range(0, top + 1, chunk):
+            bits = np.arange(lo, min(lo + chunk, top + 1), dtype=np.uint32) | np.uint32(sign)
+            x = bits.view(np.float32)
+            got, want = oracle.e4m3_encode(x), _torch_codes(x)
+            if not np.array_equal(got, want):
+                i = int(np.flatnonzero(got != want)[0])
+                raise AssertionError(f"pattern {bits[i]:#010x} ({x[i]!r}): oracle {got[i]:#04x}, "
+                                     f"torch {want[i]:#04x}")

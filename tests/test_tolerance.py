@@ -63,3 +63,20 @@ def test_scale_exponent_slip_fails():
     ws2[0, 0] *= np.float32(2.0)
     bad, _ = oracle.gemm(oracle.FPROP, xq, xs, wq, ws2)
     assert _fails(_bf16_round(bad), ref, S)
+
+
+def test_bf16_rounding_term_comes_from_the_oracle_only():
+    """The bf16 term is half a bf16 ulp of |ref| + B (B the accumulator bound): the worst
+    accumulator value rounded to bf16 passes, and anything a hair past the bound fails, whatever
+    the GPU's own magnitude."""
+    from tests._util import tolerance, ulp_bf16
+    ref = np.array([1.99, -3.999, 0.75, 1.0e-3])
+    S = np.abs(ref) * 1.5
+    B = 2e-3 * S + 1e-2 * ulp_bf16(ref)
+    bound = tolerance(ref, S, bf16_out=True)
+    assert np.allclose(bound, B + 0.5 * ulp_bf16(np.abs(ref) + B), rtol=0, atol=0)
+    worst_acc = ref + np.sign(ref) * B
+    check_gemm(_bf16_round(worst_acc), ref, S, "bf16 of the worst accumulator")
+    over = ref + np.sign(ref) * bound * (1 + 1e-9)
+    assert _fails(over, ref, S)
+    assert tolerance(ref, S, bf16_out=False).tolist() == B.tolist()
