@@ -34,6 +34,7 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 
 T_TOK, C_IN, C_OUT = 4096, 7168, 2048
+MLA_WIDTHS = (1536, 512)                         # MLA query / KV compression widths
 GEMM_FLOP = 2.0 * T_TOK * C_OUT * C_IN           # each of Fprop, Dgrad, Wgrad
 STEP_FLOP = 3.0 * GEMM_FLOP
 METRIC = ("block-scaled FP8 GEMM TFLOP/s (% dense FP8 peak); quantizer GB/s (% HBM)")
@@ -106,7 +107,7 @@ class ClockSampler:
         0x100: "display_clock_setting",
     }
 
-    def __init__(self, device_index: int, period_s: float = 0.002):
+    def __init__(self, device_index: int, period_s: float = 0.0002):
         self.samples = []
         self.reasons = set()
         self.max_mhz = None
@@ -146,11 +147,15 @@ class ClockSampler:
             self._stop.set()
             self._thread.join()
 
-    def summary(self):
+    def summary(self, steps: int | None = None):
         if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
-        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+        out = {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+               "sm_mhz_min": float(min(self.samples)), "reasons": sorted(self.reasons),
+               "samples": len(self.samples)}
+        if steps:
+            out["samples_per_step"] = round(len(self.samples) / steps, 2)
+        return out
 
 
 # ------------------------------------------------------------------------------------------ #
@@ -368,6 +373,31 @@ def run_ours(args, rank, world, dist):
             torch.cuda.synchronize()
             ts.append(e0.elapsed_time(e1))
         fused_ms[name] = round(statistics.median(ts[2:]), 5)
+    # Not part of the step either: the MLA-shaped Fprop GEMMs (query / KV down-projections,
+    # X [4096, 7168] times W [1536 | 512, 7168]^T), on the step's quantised X and their own
+    # seeded weights quantised 128x128 on the device.
+    mla = {}
+    for n_mla in MLA_WIDTHS:
+        from fp8_fine_grained_fp8q_b200 import synth
+        wm = torch.from_numpy(synth.weights(n_mla, C_IN, seed=synth.SEED_BASE + 3 + n_mla).view(np.int16)).view(
+            torch.bfloat16).to(dev)
+        wq, ws, _ = ops.weight_128x128(wm)
+        ym = torch.empty((T_TOK, n_mla), dtype=torch.bfloat16, device=dev)
+        f = lambda: ops.gemm_blockscaled(ops.FPROP, b["Xq"], b["sX"], wq, ws, ym)  # noqa: E731
+        for _ in range(3):
+            f()
+        ts = []
+        for _ in range(20):
+            flush_l2()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            f()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        mla[n_mla] = statistics.median(ts)
+    if ops.device_status(dev) != ops.DEV_OK:
+        raise RuntimeError("device status after the MLA-shaped GEMMs")
     sum_step_ms = float(sum(step_ms))
     total_ms = start.elapsed_time(end)
     sum_step_ms = max_over_ranks(sum_step_ms, dist, dev)
@@ -419,6 +449,12 @@ def run_ours(args, rank, world, dist):
             ach = amount / (ms * 1e-3) / 1e9
             kernels[name] = {"ms": round(ms, 5), "GB/s": round(ach, 1),
                              "frac_hbm": round(ach / hbm, 4)}
+    for n_mla, ms in mla.items():
+        flop = 2.0 * T_TOK * n_mla * C_IN
+        ach = flop / (ms * 1e-3) / 1e12
+        kernels[f"gemm_fprop_mla_n{n_mla}"] = {
+            "ms": round(ms, 5), "TFLOP/s": round(ach, 1), "frac_fp8_peak": round(ach / fp8_peak, 4),
+            "shape": f"{T_TOK}x{n_mla}x{C_IN}", "in_step": False}
     gemm_ms = statistics.mean([statistics.mean(per_op[n]) for n in ("gemm_fprop", "gemm_dgrad", "gemm_wgrad")])
     gemm_ach = GEMM_FLOP / (gemm_ms * 1e-3) / 1e12
     traffic = load_traffic()
@@ -450,7 +486,7 @@ def run_ours(args, rank, world, dist):
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "steps": len(e2e_ms)},
         "gpu_launches": len(launches) * args.steps,
-        "clocks": clocks.summary(),
+        "clocks": clocks.summary(args.steps),
         "wall_ms_timed_region": round(total_ms, 3),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -705,6 +741,41 @@ def run_moe(args, rank, world, dist):
     }
 
 
+def profile_moe(experts: int):
+    """One launch of the grouped MoE Fprop GEMM on the MoE workload's operands (8192 tokens x top-8
+    routed over `experts` experts), after quantising them once, for a profiler capture:
+    `-k regex:gemm_blockscaled -c 1` takes exactly that launch."""
+    import torch
+    from fp8_fine_grained_fp8q_b200 import ops, synth
+    dev = torch.device("cuda", 0)
+    expert_of, _ = synth.moe_routing(tokens=MOE_TOKENS, experts=experts, top_k=MOE_TOPK,
+                                     n_empty=max(1, experts // 32))
+    token_idx, off = synth.moe_grouped_rows(expert_of, experts)
+    mtot = int(off[-1])
+    g = torch.Generator(device=dev)
+    g.manual_seed(synth.SEED_BASE + 5)
+    x = torch.randn((MOE_TOKENS, MOE_K), device=dev, generator=g)
+    x[:, torch.randperm(MOE_K, device=dev, generator=g)[: round(0.001 * MOE_K)]] *= 100.0
+    xg = x.to(torch.bfloat16)[torch.from_numpy(token_idx).to(dev)].contiguous()
+    del x
+    wq = torch.empty((experts * MOE_N, MOE_K), dtype=torch.uint8, device=dev)
+    sw = torch.empty((experts * MOE_N // 128, MOE_K // 128), dtype=torch.float32, device=dev)
+    for e0 in range(0, experts, 32):
+        n = min(32, experts - e0)
+        w = (0.02 * torch.randn((n * MOE_N, MOE_K), device=dev, generator=g)).to(torch.bfloat16)
+        ops.weight_128x128(w, wq[e0 * MOE_N:(e0 + n) * MOE_N], sw[e0 * MOE_N // 128:(e0 + n) * MOE_N // 128])
+        del w
+    xq, sx = ops.act_1x128(xg)
+    out = torch.empty((mtot, MOE_N), dtype=torch.bfloat16, device=dev)
+    torch.cuda.synchronize()
+    ops.grouped_gemm_blockscaled(xq, sx, wq.view(experts, MOE_N, MOE_K), sw.view(experts, MOE_N // 128, MOE_K // 128),
+                                 torch.from_numpy(off).to(dev), out)
+    torch.cuda.synchronize()
+    if ops.device_status(dev) != ops.DEV_OK:
+        raise RuntimeError("device status after the grouped GEMM")
+    print(json.dumps({"profile_moe": experts, "rows": mtot, "status": "ok"}))
+
+
 def profile_gemms(fmt: str):
     """The linear layer's three GEMMs, one launch each, after one quantisation pass (for a profiler
     capture: `-k regex:gemm_blockscaled -c 3` takes exactly these launches)."""
@@ -741,7 +812,13 @@ def main():
     ap.add_argument("--profile-gemms", choices=["fp32", "ue8m0"], default=None,
                     help="no timing: quantise the layer once with this scale format, launch its Fprop, "
                          "Dgrad and Wgrad GEMMs once each and exit (a small, fixed launch list for ncu)")
+    ap.add_argument("--profile-moe", type=int, default=None, metavar="EXPERTS",
+                    help="no timing: one launch of the grouped MoE Fprop GEMM over this many experts (for a "
+                         "profiler capture) and exit")
     args = ap.parse_args()
+    if args.profile_moe:
+        profile_moe(args.profile_moe)
+        return
     if args.profile_gemms:
         profile_gemms(args.profile_gemms)
         return

@@ -384,3 +384,31 @@ def test_full_size_every_config_deterministic_and_within_tolerance(mode, cfg, mo
     assert ops.device_status() == ops.DEV_OK
     assert torch.equal(first, second)
     sampled_check(mode, a, sa, b, sb, host(first), f"mode {mode} {cfg}")
+
+
+def test_two_streams_default_workspace(monkeypatch):
+    """Two stream-K GEMMs queued on two streams at once through the default binding (no explicit
+    workspace): each stream gets its own cached workspace, so neither overwrites the other's
+    partial tiles; both results match the oracle."""
+    monkeypatch.setenv("FP8Q_GEMM_SCHED", "sk")
+    cases = []
+    for seed in (61, 62):
+        X = synth.activations_channel_outliers(1024, 2048, seed=seed)
+        W = synth.weights(768, 2048, seed=seed + 100)
+        xq, xs = oracle.quant_1x128(X)
+        wq, ws, _ = oracle.quant_128x128(W)
+        cases.append((xq, xs, wq, ws, u8_dev(xq), f32_dev(xs), u8_dev(wq), f32_dev(ws)))
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = [None, None]
+    torch.cuda.synchronize()
+    for rep in range(3):
+        for i, s in enumerate(streams):
+            with torch.cuda.stream(s):
+                *_, A, SA, B, SB = cases[i]
+                outs[i] = ops.gemm_blockscaled(FPROP, A, SA, B, SB)
+        torch.cuda.synchronize()
+        assert ops.device_status() == ops.DEV_OK
+        for i in range(2):
+            xq, xs, wq, ws = cases[i][:4]
+            ref, S = oracle.gemm(FPROP, xq, xs, wq, ws)
+            check_gemm(host(outs[i]), ref, S, f"stream {i}, repetition {rep}")
