@@ -69,7 +69,7 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-GEMM_SOURCES = ("gemm.cuh", "ptx.cuh")         # what the GEMM kernel's DRAM traffic depends on
+GEMM_SOURCES = ("fp8q.cu", "gemm.cuh", "ptx.cuh")   # the GEMM kernel and its schedule choice
 
 
 def source_hash(names=GEMM_SOURCES) -> str:
@@ -187,15 +187,20 @@ def make_buffers(torch, dev):
     return host, t, b
 
 
-def step_ops(ops, t, b, separate=False):
-    """The step as (names, zero-argument launches), all on torch's current stream.  By default
-    X and dY are quantised to both forms in one pass each (act_dual); separate=True runs the
-    1x128 and 128x1-transposed quantisers as their own launches."""
-    gemms = {
+def gemm_launches(ops, b):
+    """The linear layer's three GEMM launches on the step's buffers."""
+    return {
         "gemm_fprop": lambda: ops.gemm_blockscaled(ops.FPROP, b["Xq"], b["sX"], b["Wq"], b["sW"], b["Y"]),
         "gemm_dgrad": lambda: ops.gemm_blockscaled(ops.DGRAD, b["dYq"], b["sdY"], b["Wq"], b["sW"], b["dX"]),
         "gemm_wgrad": lambda: ops.gemm_blockscaled(ops.WGRAD, b["dYtq"], b["sdYt"], b["Xtq"], b["sXt"], b["dW"]),
     }
+
+
+def step_ops(ops, t, b, separate=False):
+    """The step as (names, zero-argument launches), all on torch's current stream.  By default
+    X and dY are quantised to both forms in one pass each (act_dual); separate=True runs the
+    1x128 and 128x1-transposed quantisers as their own launches."""
+    gemms = gemm_launches(ops, b)
     quant = {
         "quant_forward_XW": lambda: ops.quant_forward(t["X"], t["W"], b["Xq"], b["sX"], b["Xtq"], b["sXt"],
                                                       b["Wq"], b["sW"]),
@@ -289,6 +294,7 @@ def run_ours(args, rank, world, dist):
     ops.lib()                                      # fail loudly if the library is missing
     host, t, b = make_buffers(torch, dev)
     OPS, launches = step_ops(ops, t, b, separate=args.separate_quant)
+    gemm_launch = gemm_launches(ops, b)
     flush_w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     flush_r = torch.ones(64 << 20, dtype=torch.float32, device=dev)
 
@@ -376,7 +382,7 @@ def run_ours(args, rank, world, dist):
     # Not part of the step either: the MLA-shaped Fprop GEMMs (query / KV down-projections,
     # X [4096, 7168] times W [1536 | 512, 7168]^T), on the step's quantised X and their own
     # seeded weights quantised 128x128 on the device.
-    mla = {}
+    mla, mla_ops = {}, {}
     for n_mla in MLA_WIDTHS:
         from fp8_fine_grained_fp8q_b200 import synth
         wm = torch.from_numpy(synth.weights(n_mla, C_IN, seed=synth.SEED_BASE + 3 + n_mla).view(np.int16)).view(
@@ -396,8 +402,43 @@ def run_ours(args, rank, world, dist):
             torch.cuda.synchronize()
             ts.append(e0.elapsed_time(e1))
         mla[n_mla] = statistics.median(ts)
+        mla_ops[n_mla] = (wq, ws, ym)
     if ops.device_status(dev) != ops.DEV_OK:
         raise RuntimeError("device status after the MLA-shaped GEMMs")
+
+    # Each GEMM under the conditions it meets inside the step: its operands were just written (so
+    # they sit in L2) and it is launched right behind another kernel (programmatic dependent launch
+    # overlaps the two).  After an L2 flush one launch brings the operands back; then 10 launches
+    # back to back between two events; median of 7 such runs.  The per-launch breakdown above puts
+    # an event between launches instead, which serialises them and adds the launch latency to
+    # each kernel's time.
+    in_step_runs = {
+        "gemm_fprop": (gemm_launch["gemm_fprop"], GEMM_FLOP),
+        "gemm_dgrad": (gemm_launch["gemm_dgrad"], GEMM_FLOP),
+        "gemm_wgrad": (gemm_launch["gemm_wgrad"], GEMM_FLOP),
+    }
+    for n_mla, (wq, ws, ym) in mla_ops.items():
+        in_step_runs[f"gemm_fprop_mla_n{n_mla}"] = (
+            (lambda wq=wq, ws=ws, ym=ym: ops.gemm_blockscaled(ops.FPROP, b["Xq"], b["sX"], wq, ws, ym)),
+            2.0 * T_TOK * n_mla * C_IN)
+    in_step = {}
+    for name, (f, flop) in in_step_runs.items():
+        for _ in range(3):
+            f()
+        reps = []
+        for _ in range(7):
+            flush_l2()
+            f()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(10):
+                f()
+            e1.record()
+            torch.cuda.synchronize()
+            reps.append(e0.elapsed_time(e1) / 10)
+        in_step[name] = (statistics.median(reps), flop)
+    if ops.device_status(dev) != ops.DEV_OK:
+        raise RuntimeError("device status after the in-step GEMM runs")
     sum_step_ms = float(sum(step_ms))
     total_ms = start.elapsed_time(end)
     sum_step_ms = max_over_ranks(sum_step_ms, dist, dev)
@@ -455,7 +496,12 @@ def run_ours(args, rank, world, dist):
         kernels[f"gemm_fprop_mla_n{n_mla}"] = {
             "ms": round(ms, 5), "TFLOP/s": round(ach, 1), "frac_fp8_peak": round(ach / fp8_peak, 4),
             "shape": f"{T_TOK}x{n_mla}x{C_IN}", "in_step": False}
-    gemm_ms = statistics.mean([statistics.mean(per_op[n]) for n in ("gemm_fprop", "gemm_dgrad", "gemm_wgrad")])
+    kernels_in_step = {}
+    for name, (ms, flop) in in_step.items():
+        ach = flop / (ms * 1e-3) / 1e12
+        kernels_in_step[name] = {"ms": round(ms, 5), "TFLOP/s": round(ach, 1), "frac_fp8_peak": round(ach / fp8_peak, 4)}
+    gemm_ms_serial = statistics.mean([statistics.mean(per_op[n]) for n in ("gemm_fprop", "gemm_dgrad", "gemm_wgrad")])
+    gemm_ms = statistics.mean([in_step[n][0] for n in ("gemm_fprop", "gemm_dgrad", "gemm_wgrad")])
     gemm_ach = GEMM_FLOP / (gemm_ms * 1e-3) / 1e12
     traffic = load_traffic()
     roofline = {
@@ -465,6 +511,8 @@ def run_ours(args, rank, world, dist):
         "peak_source": f"{peak_kind} bf16 burst {peaks['bf16_tflops']} TFLOP/s x {FP8_OVER_BF16} "
                        "(nominal dense FP8/BF16 ratio)",
         "traffic": (traffic or {}).get("gemm_bytes_per_launch"),
+        "duration": "mean over the three GEMMs of the per-launch time under in-step conditions (kernels_in_step)",
+        "achieved_serialized": round(GEMM_FLOP / (gemm_ms_serial * 1e-3) / 1e12, 1),
     }
     q_ms = sum(statistics.mean(per_op[n]) for n in OPS if n.startswith(("act", "weight", "quant")))
     q_bytes = sum(work[n][1] for n in OPS if n.startswith(("act", "weight", "quant")))
@@ -481,6 +529,8 @@ def run_ours(args, rank, world, dist):
                        "frac_hbm": round(q_bytes / (q_ms * 1e-3) / 1e9 / hbm, 4),
                        "hbm_peak_gbs": hbm, "peak_source": peak_kind},
         "kernels": kernels,
+        "kernels_method": "events after every launch of a separate pass of the step (serialised launches)",
+        "kernels_in_step": kernels_in_step,
         "fused_output_quant_ms": fused_ms,
         "ue8m0_variant": ue8m0,
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
@@ -711,6 +761,31 @@ def run_moe(args, rank, world, dist):
             ach = amount / (ms * 1e-3) / 1e9
             kernels[name] = {"ms": round(ms, 4), "GB/s": round(ach, 1), "frac_hbm": round(ach / peaks["hbm_gbs"], 4)}
     g_ms = kernels["grouped_gemm"]["ms"]
+    # The grouped GEMM's algorithmic bytes: A codes + scales, the weights (codes + scales) of the
+    # experts that hold rows (an empty expert's weights are never read), the bf16 output.
+    live = int((counts > 0).sum())
+    g_bytes = (mtot * MOE_K * (1 + 4 / 128) + live * MOE_N * MOE_K * (1 + 4 / (128 * 128))
+               + mtot * MOE_N * 2)
+    g_gbs = g_bytes / (g_ms * 1e-3) / 1e9
+    g_tf = flop / (g_ms * 1e-3) / 1e12
+    # Roofline bound: whichever of the two floors is the longer one at these sizes.
+    t_hbm, t_tensor = g_bytes / (peaks["hbm_gbs"] * 1e9), flop / (fp8_peak * 1e12)
+    trf = load_traffic()
+    g_traffic = trf.get("moe_grouped_bytes_per_launch") if trf else None
+    if t_hbm >= t_tensor:
+        roof = {"kernel": "gemm_blockscaled_kernel (grouped)", "bound": "hbm", "achieved": round(g_gbs, 1),
+                "peak": round(peaks["hbm_gbs"], 1), "unit": "GB/s", "frac": round(g_gbs / peaks["hbm_gbs"], 4),
+                "peak_source": peak_kind, "traffic": g_traffic, "algorithmic_bytes": int(g_bytes),
+                "tensor": {"achieved": round(g_tf, 1), "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
+                           "frac": round(g_tf / fp8_peak, 4)}}
+    else:
+        roof = {"kernel": "gemm_blockscaled_kernel (grouped)", "bound": "tensor", "achieved": round(g_tf, 1),
+                "peak": round(fp8_peak, 1), "unit": "TFLOP/s", "frac": round(g_tf / fp8_peak, 4),
+                "peak_source": f"{peak_kind} bf16 burst x {FP8_OVER_BF16}", "traffic": g_traffic,
+                "algorithmic_bytes": int(g_bytes),
+                "hbm": {"achieved": round(g_gbs, 1), "peak": round(peaks["hbm_gbs"], 1), "unit": "GB/s",
+                        "frac": round(g_gbs / peaks["hbm_gbs"], 4)}}
+    roof["floors_ms"] = {"hbm": round(t_hbm * 1e3, 4), "tensor": round(t_tensor * 1e3, 4)}
     return {
         "metric": METRIC, "value": round(world * flop / (ms_per_step * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
@@ -719,10 +794,7 @@ def run_moe(args, rank, world, dist):
         "config": {"workload": MOE_WORKLOAD, "rows": mtot, "experts": MOE_E,
                    "empty_experts": int((counts == 0).sum()), "max_rows": int(counts.max()),
                    "n": MOE_N, "k": MOE_K, "l2": "flushed before every step (256 MiB write, then read)"},
-        "roofline": {"kernel": "gemm_blockscaled_kernel (grouped)", "bound": "tensor",
-                     "achieved": round(flop / (g_ms * 1e-3) / 1e12, 1), "peak": round(fp8_peak, 1),
-                     "unit": "TFLOP/s", "frac": round(flop / (g_ms * 1e-3) / 1e12 / fp8_peak, 4),
-                     "peak_source": f"{peak_kind} bf16 burst x {FP8_OVER_BF16}", "traffic": None},
+        "roofline": roof,
         "kernels": kernels,
         "grouped_dgrad": {"ms": round(dgrad_ms, 4), "TFLOP/s": round(flop / (dgrad_ms * 1e-3) / 1e12, 1),
                           "frac_fp8_peak": round(flop / (dgrad_ms * 1e-3) / 1e12 / fp8_peak, 4),

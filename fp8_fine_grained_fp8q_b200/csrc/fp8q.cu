@@ -204,14 +204,22 @@ bool streamk_forced()
     return env && strcmp(env, "sk") == 0;
 }
 
-// Stream-K pays off when the tiles do not fill whole waves of the persistent grid.
+// Stream-K pays off when the whole tiles leave the last wave of the persistent grid mostly empty;
+// otherwise its partial tiles (parked in the workspace and added by the tile's owner) and the
+// extra work items per CTA cost more than the idle SMs of the last wave.  Measured on the
+// linear-layer shapes (back-to-back launches, operands in L2): data-parallel is faster at a wave
+// occupancy of 0.865 (Fprop 4096x2048x7168: 256 tiles in 2 waves of 148; Dgrad 4096x7168x2048:
+// 896 tiles in 7), stream-K at 0.757 and below (Wgrad 2048x7168x4096: 448 tiles in 4; the MLA
+// widths 1536 and 512: 192 and 64 tiles).  The switch sits between the two, at 0.8.
 bool want_streamk(int64_t tiles, int ctas, int kb)
 {
     const char* env = getenv("FP8Q_GEMM_SCHED");
     if (env && strcmp(env, "dp") == 0) return false;
     if (kb < 2) return false;
     if (streamk_forced()) return true;
-    return tiles % ctas != 0;
+    if (tiles % ctas == 0) return false;
+    const int64_t waves = (tiles + ctas - 1) / ctas;
+    return (double)tiles < 0.8 * (double)(waves * ctas);
 }
 
 template <int MODE, int BN, bool GROUPED, bool MX = false>
