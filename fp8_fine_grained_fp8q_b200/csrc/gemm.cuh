@@ -119,7 +119,13 @@ struct GemmShape {
     static constexpr int kABytes = kBM * kBK;
     static constexpr int kBBytes = BN * kBK;
     static constexpr int kStageBytes = kABytes + kBBytes;
-    static constexpr int kStages = (BN == 256) ? 4 : 6;
+    // Wgrad keeps three stages: its promotion, not the operand feed, sets the pace, and the 48 KB
+    // freed pay for a second epilogue staging buffer per warp (the fp32 tile leaves in eight 2 KB
+    // slabs per warp; with one buffer each slab waited for the previous store to read it).
+    // Measured: linear-layer Wgrad (2048 x 7168 x 4096) 104.8 -> 100.0 us; MoE grouped Wgrad
+    // (256 experts, 65536 rows) 4.49 -> 4.17 ms.
+    static constexpr bool kWgrad3 = MODE == kModeWgrad && !MX && BN == 256;
+    static constexpr int kStages = kWgrad3 ? 3 : ((BN == 256) ? 4 : 6);
     static constexpr int kScaleStages = (MODE == kModeWgrad && !MX) ? 4 : 0;
     // MX scale factors per stage: one 512-byte chunk for A's 128 rows and one per 128 columns
     // of B.  Chunk row r (16 bytes, r = 0..31) holds the exponents of rows r, 32 + r, 64 + r,
@@ -149,7 +155,7 @@ struct GemmShape {
     // Epilogue staging: 2 KB per promotion warp and buffer, 1024-byte aligned (the 64-byte
     // swizzle of the tensor store works on absolute shared-memory address bits).  Two buffers per
     // warp where shared memory allows, so one slab's store reads while the next is written.
-    static constexpr int kEpiBufs = (MODE == kModeWgrad || GROUPED || kPW == 4 || MX) ? 1 : 2;
+    static constexpr int kEpiBufs = kWgrad3 ? 2 : ((MODE == kModeWgrad || GROUPED || kPW == 4 || MX) ? 1 : 2);
     static constexpr int kOffEpi = (kOffGroups + (GROUPED ? 2 * (kMaxGroups + 1) * 4 : 0) + 1023) / 1024 * 1024;
     static constexpr int kSmemBytes = kOffEpi + kPromoWarps * 2048 * kEpiBufs + 1024;
     // Registers (setmaxnreg moves them from the producer / MMA warpgroup to the promotion
@@ -583,9 +589,12 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
         // memory; with one row per thread each thread would need all its kCols column scales per K
         // group.  So Wgrad reads TMEM with the 16x256b shape instead: a thread holds 4 rows
         // (t/4 + 8i of the warp's 32) x 2 columns of every 8-column block, i.e. needs a quarter
-        // of the column scales (an 8-byte load per block).  Its chunk is 16 columns (16
-        // registers); acc[kBlocks * i + j] is row i's column pair of block j.
-        constexpr int kCW = (MODE == kModeWgrad || S::kCols < 32 || S::kPW == 4) ? 16 : 32;
+        // of the column scales (an 8-byte load per block).  Its chunk is 32 columns: two
+        // 16x256b.x4 loads (lanes +0 and +16) of 16 registers each, half the round trips of
+        // 16-column chunks (104.8 against 106.8 us on the linear-layer Wgrad);
+        // acc[kBlocks * i + j] is row i's column pair of block j.
+        constexpr int kCW = (S::kCols < 32 || S::kPW == 4) ? 16 : 32;
+        constexpr int kHalfW = kCW / 2;   // Wgrad: registers of one 16-lane load
         constexpr int kChunks = S::kCols / kCW;
         constexpr int kBlocks = S::kCols / 8;
         const int wt0 = lane & 3, wt1 = lane >> 2;   // Wgrad: column pair and first row of a thread
@@ -635,8 +644,8 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                         if (MODE != kModeWgrad) {
                             tmem_ld_async(taddr + ch * kCW, r);
                         } else {
-                            tmem_ld_16x256b_x2(taddr + ch * kCW, r);
-                            tmem_ld_16x256b_x2(taddr + (16u << 16) + ch * kCW, r + 8);
+                            tmem_ld_16x256b<kCW / 8>(taddr + ch * kCW, r);
+                            tmem_ld_16x256b<kCW / 8>(taddr + (16u << 16) + ch * kCW, r + kHalfW);
                         }
                     };
                     const auto take = [&](uint32_t (&cur)[kCW], int ch) {
@@ -646,13 +655,13 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                                 acc[(ch * kCW + j) / 2] = make_float2(__uint_as_float(cur[j]), __uint_as_float(cur[j + 1]));
                         } else {
 #pragma unroll
-                            for (int b = 0; b < 2; ++b)
+                            for (int b = 0; b < kCW / 8; ++b)
 #pragma unroll
                                 for (int h = 0; h < 2; ++h)
 #pragma unroll
                                     for (int q = 0; q < 2; ++q) {
-                                        const int r0 = 8 * h + 4 * b + 2 * q;
-                                        acc[kBlocks * (2 * h + q) + 2 * ch + b] =
+                                        const int r0 = kHalfW * h + 4 * b + 2 * q;
+                                        acc[kBlocks * (2 * h + q) + (kCW / 8) * ch + b] =
                                             make_float2(__uint_as_float(cur[r0]), __uint_as_float(cur[r0 + 1]));
                                     }
                         }
@@ -705,8 +714,8 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                     if (MODE != kModeWgrad) {
                         tmem_ld_async(taddr + ch * kCW, r);
                     } else {
-                        tmem_ld_16x256b_x2(taddr + ch * kCW, r);
-                        tmem_ld_16x256b_x2(taddr + (16u << 16) + ch * kCW, r + 8);
+                        tmem_ld_16x256b<kCW / 8>(taddr + ch * kCW, r);
+                        tmem_ld_16x256b<kCW / 8>(taddr + (16u << 16) + ch * kCW, r + kHalfW);
                     }
                 };
                 // Two register chunks: the TMEM load of chunk ch+1 is in flight while chunk ch is
@@ -723,16 +732,17 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                             acc[(ch * kCW + j) / 2] = __ffma2_rn(v, c2, acc[(ch * kCW + j) / 2]);
                         }
                     } else {
-                        // cur[8h + 4b + 2q + {0,1}]: row wt1 + 8q + 16h, column pair of block 2ch + b.
+                        // cur[kHalfW*h + 4b + 2q + {0,1}]: row wt1 + 8q + 16h, column pair of block
+                        // (kCW/8)*ch + b.
 #pragma unroll
-                        for (int b = 0; b < 2; ++b) {
-                            const int jb = 2 * ch + b;
+                        for (int b = 0; b < kCW / 8; ++b) {
+                            const int jb = (kCW / 8) * ch + b;
                             const float2 sc = *reinterpret_cast<const float2*>(cs + 8 * jb + 2 * wt0);
 #pragma unroll
                             for (int h = 0; h < 2; ++h) {
 #pragma unroll
                                 for (int q = 0; q < 2; ++q) {
-                                    const int i = 2 * h + q, r0 = 8 * h + 4 * b + 2 * q;
+                                    const int i = 2 * h + q, r0 = kHalfW * h + 4 * b + 2 * q;
                                     const float2 v = make_float2(__uint_as_float(cur[r0]), __uint_as_float(cur[r0 + 1]));
                                     acc[kBlocks * i + jb] = __ffma2_rn(v, __fmul2_rn(sa2w[i], sc), acc[kBlocks * i + jb]);
                                 }
