@@ -220,16 +220,18 @@ def quantised_layer():
     return _q
 
 
-def sampled_check(mode, A, sA, B, sB, got, what, seed=0):
-    M, N = got.shape
-    g = np.random.Generator(np.random.PCG64(seed))
-    rows = np.unique([0, 127, 128, M // 2 + 3, M - 1])
-    cols = np.unique([0, 127, 128, N // 2 + 5, N - 1])
-    mm = np.concatenate([np.repeat(rows, N), np.tile(np.arange(M), cols.size), g.integers(0, M, 4096)])
-    nn = np.concatenate([np.tile(np.arange(N), rows.size), np.repeat(cols, M), g.integers(0, N, 4096)])
-    ref, S = oracle.gemm_entries(mode, A, sA, B, sB, mm, nn)
+_ref = {}
+
+
+def full_check(mode, A, sA, B, sB, got, what):
+    """Every entry of a full-size result against the oracle (its exact D and S are computed once
+    per mode and shared by the configurations)."""
+    if mode not in _ref:
+        _ref[mode] = oracle.gemm(mode, A, sA, B, sB)
+    ref, S = _ref[mode]
+    assert got.shape == ref.shape
     assert np.all(np.isfinite(got)), f"{what}: unwritten or non-finite outputs"
-    return check_gemm(got[mm, nn], ref, S, what, bf16_out=(mode != WGRAD))
+    return check_gemm(got, ref, S, what, bf16_out=(mode != WGRAD))
 
 
 @pytest.mark.parametrize("cfg", ["n256-sk", "n256-dp", "n128-sk"])
@@ -243,4 +245,4 @@ def test_full_size_deterministic_and_within_tolerance(mode, cfg, monkeypatch):
     second = ops.gemm_blockscaled_ue8m0(mode, A, SA, B, SB)
     assert ops.device_status() == ops.DEV_OK
     assert torch.equal(first, second)
-    sampled_check(mode, a, sa, b, sb, host(first), f"ue8m0 mode {mode} {cfg}")
+    full_check(mode, a, sa, b, sb, host(first), f"ue8m0 mode {mode} {cfg}")
