@@ -629,7 +629,48 @@ def cpu_baseline(budget_s: float = 15.0):
     mean = statistics.mean(times)
     return {"value": round(SLICE_FLOP / mean / 1e12, 6), "unit": "TFLOP/s",
             "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": SLICE_DESC + f"; {len(times)} repetitions, {sum(times):.1f} s"}
+            "sample": SLICE_DESC + f"; {len(times)} repetitions, {sum(times):.1f} s",
+            "quantizers": cpu_quantizers(oracle)}
+
+
+def cpu_quantizers(oracle, budget_s: float = 2.0):
+    """The oracle's three quantisers on 512 tokens of X [., 7168] (both activation forms) and
+    256 rows of W [., 7168], as algorithmic GB/s, on one thread and on all cores."""
+    import ctypes
+    from fp8_fine_grained_fp8q_b200 import synth
+    d = synth.linear_layer(T_TOK, C_IN, C_OUT)
+    x, w = np.ascontiguousarray(d["X"][:512]), np.ascontiguousarray(d["W"][:256])
+    nbytes = 2 * x.size * QB_1x128 + w.size * QB_128x128
+
+    def run():
+        oracle.quant_1x128(x)
+        oracle.quant_128x1_t(x)
+        oracle.quant_128x128(w)
+
+    def rate():
+        run()
+        n, t0 = 0, time.perf_counter()
+        while n < 2 or time.perf_counter() - t0 < budget_s:
+            run()
+            n += 1
+        return nbytes * n / (time.perf_counter() - t0) / 1e9
+
+    out = {"unit": "GB/s", "sample": "X [512, 7168] to 1x128 and 128x1-transposed, W [256, 7168] to 128x128 "
+                                     f"({nbytes / 1e6:.1f} MB of algorithmic traffic per pass)"}
+    cores = oracle.num_threads()
+    out["all_cores"], out["cores"] = round(rate(), 3), cores
+    out["one_thread"] = None
+    try:
+        gomp = ctypes.CDLL("libgomp.so.1")      # the OpenMP runtime the oracle's library runs on
+    except OSError:
+        return out
+    gomp.omp_set_num_threads(1)
+    try:
+        if oracle.num_threads() == 1:
+            out["one_thread"] = round(rate(), 3)
+    finally:
+        gomp.omp_set_num_threads(cores)
+    return out
 
 
 def run_reference(args, rank, world):
