@@ -107,7 +107,7 @@ class ClockSampler:
         0x100: "display_clock_setting",
     }
 
-    def __init__(self, device_index: int, period_s: float = 0.0002):
+    def __init__(self, device_index: int, period_s: float = 0.0):
         self.samples = []
         self.reasons = set()
         self.max_mhz = None
@@ -124,28 +124,34 @@ class ClockSampler:
             self._nvml = None
 
     def _run(self):
+        # The SM clock on every pass, the event reasons on every fourth: one NVML query takes
+        # 0.1-0.2 ms, and a timed step lasts ~0.3 ms, so the clock gets a sample (or more) per step.
         nv = self._nvml
+        n = 0
         while not self._stop.is_set():
             try:
                 self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
-                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
-                for bit, name in self.REASONS.items():
-                    if mask & bit and bit != 0x1:
-                        self.reasons.add(name)
+                if n % 4 == 0:
+                    mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                    for bit, name in self.REASONS.items():
+                        if mask & bit and bit != 0x1:
+                            self.reasons.add(name)
             except Exception:
                 pass
-            time.sleep(self.period)
+            n += 1
+            if self.period > 0:
+                time.sleep(self.period)
+
+    def __exit__(self, *exc):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
 
     def __enter__(self):
         if self._nvml is not None:
             self._thread = threading.Thread(target=self._run, daemon=True)
             self._thread.start()
         return self
-
-    def __exit__(self, *exc):
-        if self._thread is not None:
-            self._stop.set()
-            self._thread.join()
 
     def summary(self, steps: int | None = None):
         if not self.samples:
