@@ -21,6 +21,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -72,13 +73,23 @@ def load_peaks():
 GEMM_SOURCES = ("fp8q.cu", "gemm.cuh", "ptx.cuh")   # the GEMM kernel and its schedule choice
 
 
+def code_only(text: str) -> str:
+    """C/C++ source without its comments, trailing blanks and blank lines (string literals that
+    contain comment markers do not occur in the hashed files)."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
 def source_hash(names=GEMM_SOURCES) -> str:
+    """Hash of the GEMM sources' code (comments excluded): the DRAM counters in
+    profiles/traffic.json describe the kernel built from exactly this code."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "fp8_fine_grained_fp8q_b200", "csrc")
     for name in sorted(names):
-        with open(os.path.join(csrc, name), "rb") as f:
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
             h.update(name.encode())
-            h.update(f.read())
+            h.update(code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -139,7 +139,8 @@ struct GemmShape {
     // Promotion warpgroups.  Each owns BN / kPW columns of the tile (all 128 rows; warp w of a
     // group reads TMEM lanes 32*(w%4) ..).  Two: four groups (640 threads) halve each thread's
     // arithmetic per K group but not its TMEM round trips, which set the fold's length; with
-    // 104 registers per thread they measured 6-8 % slower on the linear-layer shapes.
+    // 104 registers per thread they measured 6-8 % slower on the linear-layer Fprop / Dgrad and
+    // 43 % slower on Wgrad (whose fold then spills).
     static constexpr int kPW = 2;
     static constexpr int kPromoWarps = 4 * kPW;
     static constexpr int kPromoThreads = 128 * kPW;
