@@ -589,9 +589,13 @@ def run_ours(args, rank, world, dist):
                    "l2": "flushed before every step, outside the step: 256 MiB write, then 256 MiB read of another buffer",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "roofline": roofline,
-        "quantizers": {"GB/s": round(q_bytes / (q_ms * 1e-3) / 1e9, 1),
-                       "frac_hbm": round(q_bytes / (q_ms * 1e-3) / 1e9 / hbm, 4),
-                       "hbm_peak_gbs": hbm, "peak_source": peak_kind},
+        "quantizers": {"GB/s": quantizers_device["aggregate"]["GB/s"],
+                       "frac_hbm": quantizers_device["aggregate"]["frac_hbm"],
+                       "hbm_peak_gbs": hbm, "peak_source": peak_kind,
+                       "method": "the step's quantiser launches, device time (quantizers_device)",
+                       "serialized": {"GB/s": round(q_bytes / (q_ms * 1e-3) / 1e9, 1),
+                                      "frac_hbm": round(q_bytes / (q_ms * 1e-3) / 1e9 / hbm, 4),
+                                      "method": "events around each launch of a separate pass (kernels)"}},
         "quantizers_device": quantizers_device,
         "kernels": kernels,
         "kernels_method": "events after every launch of a separate pass of the step (serialised launches)",

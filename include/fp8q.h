@@ -171,8 +171,9 @@ FP8Q_API int fp8q_weight_128x128(const uint16_t* w, int64_t N, int64_t K, uint8_
  * Requirements: K % 128 == 0, N % 128 == 0 (FP8Q_ERR_SHAPE); M >= 0 (any M, the last row tile
  * is masked); M, N, K < 2^31 (FP8Q_ERR_UNSUPPORTED).  D is fully overwritten, except in
  * FP8Q_WGRAD_ACC.  K == 0 writes D = 0 (FP8Q_WGRAD_ACC: leaves D unchanged).
- * workspace / ws_bytes: optional scratch for the stream-K schedule (used when the output tiles do
- * not fill whole waves of the persistent grid): at least fp8q_gemm_workspace_size(...) bytes,
+ * workspace / ws_bytes: optional scratch for the stream-K schedule (used when whole output tiles
+ * would leave the persistent grid's last wave less than 80 % full, and K spans at least two
+ * 128-groups): at least fp8q_gemm_workspace_size(...) bytes,
  * 256-byte aligned, device memory owned by the caller, reusable across calls on one stream
  * (never cleared: each launch stamps its flags with a fresh value).  NULL / 0, or a smaller
  * buffer, runs the data-parallel schedule instead -- same results, possibly slower.
