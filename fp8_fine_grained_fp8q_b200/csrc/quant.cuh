@@ -152,16 +152,16 @@ __global__ void __launch_bounds__(256) act_1x128_kernel(const uint16_t* __restri
 template <int kSh>
 __device__ __forceinline__ int qt_unit(int row, int u) { return row * 8 + (u ^ ((row >> kSh) & 7)); }
 
-// Rows [row0, row0 + 4 * n) of a staged code tile, 4 rows per warp instruction, to qt (row pitch
-// pitch bytes, first token column col0).
-__device__ __forceinline__ void qt_store_rows(const uint4* qs, int kSh_is_2, int row0, int n,
-                                              uint8_t* __restrict__ qt, int64_t c0, int64_t pitch,
-                                              int64_t col0, int lane)
+// Rows [row0, row0 + 4 * N) of a staged code tile (laid out by qt_unit<kSh>), 4 rows per warp
+// instruction, to qt (row pitch `pitch` bytes, first token column col0).
+template <int kSh, int N>
+__device__ __forceinline__ void qt_store_rows(const uint4* qs, int row0, uint8_t* __restrict__ qt, int64_t c0,
+                                              int64_t pitch, int64_t col0, int lane)
 {
-    for (int k = 0; k < n; ++k) {
+#pragma unroll
+    for (int k = 0; k < N; ++k) {
         const int row = row0 + 4 * k + (lane >> 3), u = lane & 7;
-        const int idx = kSh_is_2 ? qt_unit<2>(row, u) : qt_unit<1>(row, u);
-        *reinterpret_cast<uint4*>(qt + (c0 + row) * pitch + col0 + 16 * u) = qs[idx];
+        *reinterpret_cast<uint4*>(qt + (c0 + row) * pitch + col0 + 16 * u) = qs[qt_unit<kSh>(row, u)];
     }
 }
 
@@ -220,7 +220,7 @@ __global__ void __launch_bounds__(256) act_128x1_t_kernel(const uint16_t* __rest
     qs[qt_unit<1>(2 * lane, w)] = make_uint4(q0[0], q0[1], q0[2], q0[3]);
     qs[qt_unit<1>(2 * lane + 1, w)] = make_uint4(q1[0], q1[1], q1[2], q1[3]);
     __syncthreads();
-    qt_store_rows(qs, 0, 8 * w, 2, qt, c0, T, t0, lane);
+    qt_store_rows<1, 2>(qs, 8 * w, qt, c0, T, t0, lane);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -336,7 +336,7 @@ __global__ void __launch_bounds__(256) act_128x1_t_ragged_kernel(const uint16_t*
         qs[qt_unit<1>(2 * lane, w)] = make_uint4(q0[0], q0[1], q0[2], q0[3]);
         qs[qt_unit<1>(2 * lane + 1, w)] = make_uint4(q1[0], q1[1], q1[2], q1[3]);
         __syncthreads();
-        qt_store_rows(qs, 0, 8 * w, 2, qt, c0, Kcap, (int64_t)g * 128, lane);
+        qt_store_rows<1, 2>(qs, 8 * w, qt, c0, Kcap, (int64_t)g * 128, lane);
         __syncthreads();   // red, inv_c and qs are rewritten by the next channel block
     }
 }
@@ -451,7 +451,7 @@ __device__ __forceinline__ void act_dual_tile(const uint16_t* __restrict__ x, ui
 #pragma unroll
     for (int j = 0; j < 4; ++j) qs[qt_unit<2>(4 * lane + j, w)] = make_uint4(c[j][0], c[j][1], c[j][2], c[j][3]);
     __syncthreads();
-    qt_store_rows(qs, 1, 16 * w, 4, qt, c0, T, t0, lane);
+    qt_store_rows<2, 4>(qs, 16 * w, qt, c0, T, t0, lane);
 }
 
 template <bool POW2>
